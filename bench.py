@@ -1,0 +1,315 @@
+#!/usr/bin/env python
+"""Throughput of the quantized attention forward on B200.
+
+One step = one pass of the whole hot path over one batch: smoothing + INT8/FP8
+quantization of Q, K, V (libsage quantize kernels) and the fused attention
+kernel, all through the C ABI (libsage.so).
+
+Default workload: LLM prefill, B1 H32 N8192 d128 bf16, causal, INT8 QK / FP8 PV
+(FP32 accumulator).  Inputs (192 MB of bf16 Q, K, V) are larger than the 126 MB
+L2, so no flush runs between steps.
+
+Prints ONE JSON line (rank 0).  `value` is whole-job attention TOPS counted over
+the (query, key) pairs the mask leaves visible (causal: N(N+1)/2 pairs);
+`value_square_count` is the same time with 4*B*H*N^2*d.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun each rank runs its own copy of the workload (independent
+(b, h) slices, no collective on the data path): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import signal
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_attention_sub_b200 import api, inputs  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0   # nominal dense ratio 4.5 / 2.25 PFLOP/s (INT8 dense equals FP8 dense)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(w, max_rows):
+    """The CPU oracle as it stands on a bounded sample of the workload: slice
+    (b=0, h=0) quantized in full, attention for `max_rows` evenly spaced
+    query rows.  Returns (ops of the sampled rows, seconds, threads)."""
+    import oracle as orc
+    q, k, v = inputs.generate(inputs.variant(w, B=1, H=1))
+    f = lambda t: t.float().reshape(1, w.N, w.d).numpy()
+    rows = np.unique(np.linspace(0, w.N - 1, min(max_rows, w.N)).astype(np.int32))
+    t0 = time.perf_counter()
+    qz = orc.quantize_int8_fp8(f(q), f(k), f(v), smooth_q=w.smooth_q, mode=w.mode)
+    orc.attention_int8_fp8(qz, w.causal, rows=rows)
+    dt = time.perf_counter() - t0
+    keys = (rows.astype(np.float64) + 1) if w.causal else np.full(len(rows), float(w.N))
+    ops = float(4.0 * w.d * keys.sum())
+    return ops, dt, orc.num_threads(), len(rows)
+
+
+def run_reference(args, w, ws, rank):
+    if rank != 0:
+        return
+    import oracle as orc
+    orc.build()
+    rows = 512
+    for _ in range(args.warmup):
+        oracle_sample(w, rows)
+    tot_ops, tot_t, thr, nr = 0.0, 0.0, 1, rows
+    for _ in range(args.steps):
+        ops, dt, thr, nr = oracle_sample(w, rows)
+        tot_ops += ops
+        tot_t += dt
+    value = tot_ops / tot_t / 1e12
+    sample = "slice (b0,h0) of %s quantized in full + attention of %d evenly spaced query rows per step" % (w.name, nr)
+    line = {"impl": "reference", "metric": "attention TOPS (visible-pair count)", "value": value,
+            "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8/fp8 codes, fp32 arithmetic", "data": "synthetic",
+            "config": config_of(w, args, ws),
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": thr, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args, ws):
+    return {"workload": w.name, "B": w.B * ws, "H": w.H, "N": w.N, "d": w.d, "dtype": w.dtype,
+            "causal": w.causal, "mode": ["INT8_FP8", "INT8_FP8_F16ACC", "NVFP4"][w.mode], "smooth_q": w.smooth_q,
+            "parallelism": "replicas x%d (independent (b,h) slices per rank)" % ws,
+            "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no flush" % (
+                w.B * w.H * w.N * w.d * 2 / 1e6)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llm_prefill")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    w = inputs.WORKLOADS[args.workload] if args.workload in inputs.WORKLOADS else None
+    if w is None and args.workload.startswith("sweep_"):
+        _, n, d, c = args.workload.split("_")
+        w = inputs.sweep(int(n[1:]), int(d[1:]), c == "causal")
+    ws, rank, local = dist_init() if args.impl == "ours" or int(os.environ.get("WORLD_SIZE", "1")) > 1 else (1, 0, 0)
+
+    if args.impl == "reference":
+        run_reference(args, w, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, N, d = w.shape()
+    dcode = api.DTYPE_CODE[inputs.DTYPES[w.dtype]]
+    # each rank draws its own slice batch (seed offset by rank)
+    wr = inputs.variant(w, seed=w.seed + 7919 * rank)
+    q, k, v = [t.to(dev) for t in inputs.generate(wr, device="cuda")]
+    out = torch.empty_like(q)
+    wsbuf = api.alloc_workspace(B, H, N, d, w.mode, dev)
+    nbytes = wsbuf.numel()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.sage_quantize_qkv(q, k, v, dcode, B, H, N, d, w.smooth_q, w.mode, wsbuf, nbytes, stream)
+        ev_a.record(stream)
+        api.sage_attn_quantized(wsbuf, nbytes, out, dcode, B, H, N, d, w.causal, w.smooth_q, w.mode, stream)
+        ev_b.record(stream)
+
+    ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        step()
+    api.sage_check(wsbuf, nbytes, stream)
+
+    # timed region: K steps; per-step attention-kernel events on the launch stream
+    attn_ms = []
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev_a, ev_b = ev_pairs[i]
+        step()
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    api.sage_check(wsbuf, nbytes, stream)
+    ms = t_start.elapsed_time(t_stop) / args.steps
+    attn_ms = [a_.elapsed_time(b_) for a_, b_ in ev_pairs]
+    ms = allreduce_max(ms, ws)
+    attn_avg = allreduce_max(float(np.mean(attn_ms)), ws)
+
+    ops_visible = inputs.executed_ops(w) * ws
+    ops_square = inputs.attention_ops(w) * ws
+    value = ops_visible / (ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (attention), live CUDA-event time
+    peaks, peak_src = load_peaks()
+    peak_fp8 = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    achieved = inputs.executed_ops(w) / (attn_avg * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_i8f8_kernel", "achieved": achieved, "peak": peak_fp8,
+                "unit": "TFLOP/s", "frac": achieved / peak_fp8,
+                "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense FP8/INT8 : BF16 ratio)" % (
+                    peak_src, FP8_OVER_BF16),
+                "traffic": None, "attn_ms": attn_avg}
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the region
+    hq, hk, hv = [t.cpu().pin_memory() for t in (q, k, v)]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        api.sage_attn_fwd(dq, dk, dv, out, B, H, N, d, w.causal, w.mode, dcode, w.smooth_q, wsbuf, nbytes, stream)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allreduce_max(e0.elapsed_time(e1) / e2e_steps, ws)
+    api.sage_check(wsbuf, nbytes, stream)
+    in_bytes = 3 * q.numel() * q.element_size()
+    out_bytes = out.numel() * out.element_size()
+
+    line = {"metric": "attention TOPS (4*B*H*d per visible (query,key) pair / time)", "value": value,
+            "unit": "TOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 QK / e4m3 PV, fp32 softmax and accumulation", "data": "synthetic",
+            "config": config_of(w, args, ws),
+            "value_square_count": ops_square / (ms * 1e-3) / 1e12,
+            "roofline": roofline,
+            "e2e": {"value": ops_visible / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes},
+            "gpu_launches": 6 * args.steps,
+            "clocks": clk}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle as orc
+        orc.build()
+        ops, dt, thr, nr = oracle_sample(w, 2048)
+        line["cpu_baseline"] = {"value": ops / dt / 1e12, "unit": "TOPS", "cores": thr, "kind": "oracle",
+                                "sample": "slice (b0,h0) quantized in full + attention of %d evenly spaced "
+                                          "query rows; %.1f s" % (nr, dt)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

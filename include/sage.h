@@ -1,0 +1,148 @@
+/*
+ * sage.h -- C ABI of libsage.so, the B200 (sm_100a) SageAttention-family
+ * quantized attention forward.
+ *
+ * The operation (citations are to the pages this library follows):
+ *   - SageAttention2 Technical Report, abstract: smooth the inputs, quantize
+ *     Q and K to low-bit integers at a fine (warp-level) granularity and
+ *     (P~, V) to FP8, then run attention on the quantized operands.
+ *   - SageAttention2++ summary, Sec. 2.1: Q and K (and P~) carry per-block
+ *     scale factors, V a per-channel scale; Sec. 2: the kernel is
+ *     FlashAttention-based (tiled, online softmax); Sec. 3: the PV matmul may
+ *     accumulate in FP16 with P and V ranges narrowed to Pr = 224, Vr = 4.5
+ *     (Sec. 3.1), two MMA results summed in FP16 before FP32 (Sec. 3.2).
+ *   - SageAttention3 abstract: microscaling FP4 attention on Blackwell.
+ * INT4 QK of the pages is INT8 here: sm_100a tcgen05 has no INT4 MMA.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are contiguous row-major [B, H, N, d] in fp16 or bf16 device
+ *     memory; self-attention (query and key length N); softmax scale 1/sqrt(d).
+ *   - The caller owns all device memory (inputs, output, workspace) and the
+ *     stream.  The library never allocates, frees or synchronizes, except
+ *     sage_check, which synchronizes the given stream.
+ *   - All work is enqueued asynchronously on `stream` (0 = legacy default).
+ *   - Supported: d in {64, 128}, N >= 1, B*H >= 1, B*H*Npad*d < 2^31 where
+ *     Npad = ceil(N / 128) * 128.  Other values return SAGE_ERR_UNSUPPORTED
+ *     or SAGE_ERR_INVALID_ARG before any launch; a launch failure returns
+ *     SAGE_ERR_CUDA.  sage_last_error() gives a message for the last non-OK
+ *     status of the calling thread.
+ *   - The kernels never trap.  Every wait inside them is bounded; a wait that
+ *     runs out records an error word in the workspace and the kernel returns.
+ *     sage_check() reports it as SAGE_ERR_TIMEOUT.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAGE_API __attribute__((visibility("default")))
+#else
+#define SAGE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sage_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,
+  SAGE_ERR_UNSUPPORTED = 2,
+  SAGE_ERR_CUDA = 3,
+  SAGE_ERR_TIMEOUT = 4
+} sage_status;
+
+/* INT8 QK + FP8 PV with FP32 accumulation (SageAttention2, Sec. 2.1);
+ * the same with the FP16 PV accumulator (SageAttention2++, Sec. 3);
+ * microscaled FP4 (SageAttention3). */
+typedef enum { SAGE_MODE_INT8_FP8 = 0, SAGE_MODE_INT8_FP8_F16ACC = 1, SAGE_MODE_NVFP4 = 2 } sage_mode;
+
+typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype;
+
+/* Byte offsets into the workspace of each quantized buffer (INT8/FP8 modes).
+ * Npad = ceil(N/128)*128, BH = B*H.  Every offset is 1024-byte aligned.
+ *   q_codes  int8  [BH, Npad, d]   Q codes, one granule = 32 tokens; pad rows 0
+ *   k_codes  int8  [BH, Npad, d]   smoothed K codes, one granule = 64 tokens
+ *   vt_codes uint8 [BH, d, Npad]   e4m3 V codes, transposed (token-contiguous)
+ *   q_scale  f32   [BH, Npad/32]   per-granule scale (absmax / 127), 0 for empty
+ *   k_scale  f32   [BH, Npad/64]
+ *   v_scale  f32   [BH, d]         per-channel scale absmax / Vr
+ *   k_mean   f32   [BH, d]         per-channel mean of K over the N tokens
+ *   q_mean   f32   [BH, d]         same for Q (written only when smooth_q)
+ *   q_bias   f32   [BH, Npad]      sum_c q_mean[c] * (k - k_mean)[n, c] (smooth_q)
+ *   error    int32 (one word)      0, or the code of a wait that ran out
+ *   scratch  f32                   partial sums of the statistics pass
+ * In the NVFP4 mode q/k/vt_codes hold two e2m1 codes per byte (low nibble =
+ * even index) with sizes halved along d (Q, K) or tokens (V^T); q/k/v_scale
+ * hold ue4m3 block scales [BH,Npad,d/16], [BH,Npad,d/16], [BH,d,Npad/16];
+ * global_scale holds fp32 [BH, 3] (Q, K, V). */
+typedef struct {
+  size_t q_codes, k_codes, vt_codes, q_scale, k_scale, v_scale;
+  size_t k_mean, q_mean, q_bias, global_scale, error, scratch;
+  size_t total;
+} sage_ws_layout;
+
+/* Fill `out` with the workspace layout for a problem; returns its size in
+ * out->total.  Pure host computation. */
+SAGE_API sage_status sage_workspace_layout(int B, int H, int N, int d, int mode, sage_ws_layout* out);
+
+/* Workspace bytes needed (0 if the arguments are unsupported). */
+SAGE_API size_t sage_workspace_size(int B, int H, int N, int d, int mode);
+
+/* Smoothing + quantization (SageAttention2 abstract; SageAttention2++ Sec.
+ * 2.1, 3.1): K minus its per-channel mean over tokens; if smooth_q, Q minus
+ * its mean and the bias mean_q . (k - mean_k) per key; INT8 Q (32-token
+ * granules) and K (64-token granules) with scale absmax/127 and codes
+ * round-to-nearest-even of x * (127/absmax); V to e4m3 per channel with
+ * scale absmax/Vr (Vr = 448, or 4.5 in SAGE_MODE_INT8_FP8_F16ACC), stored
+ * transposed.  q, k, v: device [B,H,N,d] of `dtype`.  ws: device workspace of
+ * at least sage_workspace_size() bytes, 1024-byte aligned. */
+SAGE_API sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
+                              int smooth_q, int mode, void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* Fused attention on a workspace filled by sage_quantize_qkv with the same
+ * (B,H,N,d,smooth_q,mode): per 128-query tile, for each 128-key tile, INT8
+ * QK^T on the tensor cores, dequantize (scale_q * scale_k, plus the Q bias),
+ * online softmax in base 2, P~ = e4m3(p * Pr) with Pr = 448 (224 in the F16ACC
+ * mode), FP8 P~ V, and O = acc * scale_v / (Pr * l) (SageAttention2++ Sec. 2,
+ * 2.1, 3).  causal masks key j > query i.  out: device [B,H,N,d] of `dtype`. */
+SAGE_API sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
+                                int causal, int smooth_q, int mode, sage_stream_t stream);
+
+/* sage_quantize_qkv followed by sage_attn_quantized: the drop-in attention
+ * call ("plug-and-play", SageAttention2 abstract). */
+SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                          int causal, int mode, int dtype, int smooth_q, void* ws, size_t ws_bytes,
+                          sage_stream_t stream);
+
+/* Parity helper: the INT32 tile S = Q^ K^T of query tile `q_tile` and key tile
+ * `k_tile` (128 x 128) of slice `bh`, computed by the same tensor-core path as
+ * the attention kernel (kind::i8 MMA, accumulator in TMEM).  out: device
+ * int32 [128, 128], row = query.  INT8 modes only. */
+SAGE_API sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,
+                              int k_tile, int32_t* out, sage_stream_t stream);
+
+/* Test helper for the failure path: launches one thread that waits on a
+ * barrier nothing completes.  The bounded wait gives up after about 2 s, sets
+ * the workspace error word, and the kernel returns; the CUDA context stays
+ * usable.  A following sage_check() returns SAGE_ERR_TIMEOUT.  Uses only the
+ * error word at offset 0 of `ws` (>= 4 bytes, 1024-byte aligned). */
+SAGE_API sage_status sage_debug_timeout_probe(void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* Synchronize `stream`, then read and clear the workspace error word.
+ * Returns SAGE_ERR_TIMEOUT if a kernel gave up a wait, SAGE_ERR_CUDA on a
+ * CUDA error, else SAGE_OK. */
+SAGE_API sage_status sage_check(void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+SAGE_API const char* sage_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_H_ */

@@ -1,0 +1,171 @@
+"""Thin Python binding of libsage.so (include/sage.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+passes torch tensors' device pointers and the current CUDA stream through
+ctypes.  There is no fallback: if the library is missing, or a call returns a
+non-OK status, a RuntimeError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage.so")
+
+SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIMEOUT = range(5)
+MODE_INT8_FP8, MODE_INT8_FP8_F16ACC, MODE_NVFP4 = 0, 1, 2
+DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
+
+EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_attn_quantized",
+            "sage_attn_fwd", "sage_debug_qk_s32", "sage_debug_timeout_probe", "sage_check", "sage_last_error")
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("q_codes", "k_codes", "vt_codes", "q_scale", "k_scale", "v_scale",
+                                               "k_mean", "q_mean", "q_bias", "global_scale", "error", "scratch",
+                                               "total")]
+
+
+class SageError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("sage status %d: %s" % (status, message))
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsage.so (built in-tree by quantized_attention_sub_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libsage.so is not built (run __graft_entry__.build() or "
+                               "python -m quantized_attention_sub_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        i, sz, vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+        L.sage_workspace_layout.argtypes = [i, i, i, i, i, ctypes.POINTER(WsLayout)]
+        L.sage_workspace_layout.restype = i
+        L.sage_workspace_size.argtypes = [i, i, i, i, i]
+        L.sage_workspace_size.restype = sz
+        L.sage_quantize_qkv.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_quantize_qkv.restype = i
+        L.sage_attn_quantized.argtypes = [vp, sz, vp, i, i, i, i, i, i, i, i, vp]
+        L.sage_attn_quantized.restype = i
+        L.sage_attn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_attn_fwd.restype = i
+        L.sage_debug_qk_s32.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
+        L.sage_debug_qk_s32.restype = i
+        L.sage_debug_timeout_probe.argtypes = [vp, sz, vp]
+        L.sage_debug_timeout_probe.restype = i
+        L.sage_check.argtypes = [vp, sz, vp]
+        L.sage_check.restype = i
+        L.sage_last_error.argtypes = []
+        L.sage_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _raise(st):
+    if st != SAGE_OK:
+        raise SageError(st, lib().sage_last_error().decode())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+# ------------------------------------------------------------------ C names
+def sage_workspace_layout(B, H, N, d, mode) -> WsLayout:
+    out = WsLayout()
+    _raise(lib().sage_workspace_layout(B, H, N, d, mode, ctypes.byref(out)))
+    return out
+
+
+def sage_workspace_size(B, H, N, d, mode) -> int:
+    return lib().sage_workspace_size(B, H, N, d, mode)
+
+
+def sage_quantize_qkv(q, k, v, dtype, B, H, N, d, smooth_q, mode, ws, ws_bytes, stream=None):
+    _raise(lib().sage_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), dtype, B, H, N, d, int(smooth_q), mode, _ptr(ws),
+                                   ws_bytes, _stream(stream)))
+
+
+def sage_attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream=None):
+    _raise(lib().sage_attn_quantized(_ptr(ws), ws_bytes, _ptr(out), dtype, B, H, N, d, int(causal), int(smooth_q),
+                                     mode, _stream(stream)))
+
+
+def sage_attn_fwd(q, k, v, out, B, H, N, d, causal, mode, dtype, smooth_q, ws, ws_bytes, stream=None):
+    _raise(lib().sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, int(causal), mode, dtype,
+                               int(smooth_q), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def sage_debug_qk_s32(ws, ws_bytes, B, H, N, d, bh, q_tile, k_tile, out, stream=None):
+    _raise(lib().sage_debug_qk_s32(_ptr(ws), ws_bytes, B, H, N, d, bh, q_tile, k_tile, _ptr(out), _stream(stream)))
+
+
+def sage_debug_timeout_probe(ws, ws_bytes, stream=None):
+    _raise(lib().sage_debug_timeout_probe(_ptr(ws), ws_bytes, _stream(stream)))
+
+
+def sage_check(ws, ws_bytes, stream=None):
+    _raise(lib().sage_check(_ptr(ws), ws_bytes, _stream(stream)))
+
+
+# ------------------------------------------------------------------ torch helpers
+def alloc_workspace(B, H, N, d, mode, device="cuda") -> torch.Tensor:
+    """A device byte tensor big enough for the problem (torch's allocator
+    returns blocks aligned to at least 512 bytes; the library needs 1024, so
+    one extra KiB is taken and the view is offset)."""
+    n = sage_workspace_size(B, H, N, d, mode)
+    if n == 0:
+        _raise(lib().sage_workspace_layout(B, H, N, d, mode, ctypes.byref(WsLayout())))
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 1024
+    return raw[off:off + n]
+
+
+def ws_views(ws: torch.Tensor, B, H, N, d, mode) -> dict:
+    """Typed views of the quantized buffers inside a workspace (INT8/FP8 modes)."""
+    L = sage_workspace_layout(B, H, N, d, mode)
+    BH, Np = B * H, (N + 127) // 128 * 128
+
+    def view(off, nbytes, dtype, shape):
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    return dict(
+        q_codes=view(L.q_codes, BH * Np * d, torch.int8, (BH, Np, d)),
+        k_codes=view(L.k_codes, BH * Np * d, torch.int8, (BH, Np, d)),
+        vt_codes=view(L.vt_codes, BH * d * Np, torch.uint8, (BH, d, Np)),
+        q_scale=view(L.q_scale, BH * (Np // 32) * 4, torch.float32, (BH, Np // 32)),
+        k_scale=view(L.k_scale, BH * (Np // 64) * 4, torch.float32, (BH, Np // 64)),
+        v_scale=view(L.v_scale, BH * d * 4, torch.float32, (BH, d)),
+        k_mean=view(L.k_mean, BH * d * 4, torch.float32, (BH, d)),
+        q_mean=view(L.q_mean, BH * d * 4, torch.float32, (BH, d)),
+        q_bias=view(L.q_bias, BH * Np * 4, torch.float32, (BH, Np)),
+    )
+
+
+def attn_fwd(q, k, v, causal=False, mode=MODE_INT8_FP8, smooth_q=False, out=None, ws=None, stream=None):
+    """Quantized attention of [B,H,N,d] fp16/bf16 CUDA tensors (one library call)."""
+    B, H, N, d = q.shape
+    for t in (q, k, v):
+        if not (t.is_cuda and t.is_contiguous() and t.shape == q.shape and t.dtype == q.dtype):
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    if q.dtype not in DTYPE_CODE:
+        raise ValueError("dtype must be float16 or bfloat16")
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = alloc_workspace(B, H, N, d, mode, q.device)
+    sage_attn_fwd(q, k, v, out, B, H, N, d, causal, mode, DTYPE_CODE[q.dtype], smooth_q, ws, ws.numel(), stream)
+    return out

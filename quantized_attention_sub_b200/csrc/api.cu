@@ -1,0 +1,251 @@
+// api.cu -- the C ABI of libsage.so (declared in include/sage.h): argument
+// checks, workspace layout, tensor-map encoding and kernel launches.
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "../../include/sage.h"
+#include "sage_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sage_status set_err(sage_status st, const char* fmt, const char* detail = "") {
+  char buf[512];
+  snprintf(buf, sizeof(buf), fmt, detail);
+  g_last_error = buf;
+  return st;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr size_t kAlign = 1024;
+
+sage_status check_shape(int B, int H, int N, int d, int mode) {
+  if (B < 1 || H < 1 || N < 1) return set_err(SAGE_ERR_INVALID_ARG, "B, H and N must be >= 1%s");
+  if (d != 64 && d != 128) return set_err(SAGE_ERR_UNSUPPORTED, "head dimension must be 64 or 128%s");
+  if (mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_INT8_FP8_F16ACC && mode != SAGE_MODE_NVFP4)
+    return set_err(SAGE_ERR_INVALID_ARG, "unknown mode%s");
+  const long long npad = ((long long)N + 127) / 128 * 128;
+  if ((long long)B * H * npad * d >= (1LL << 31) || (long long)B * H > 65535)
+    return set_err(SAGE_ERR_UNSUPPORTED, "problem too large (B*H*Npad*d must be < 2^31, B*H <= 65535)%s");
+  return SAGE_OK;
+}
+
+sage_ws_layout layout_of(int B, int H, int N, int d, int mode) {
+  sage_ws_layout L;
+  memset(&L, 0, sizeof(L));
+  const size_t BH = (size_t)B * H, Np = ((size_t)N + 127) / 128 * 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  L.error = take(sizeof(int));
+  if (mode == SAGE_MODE_NVFP4) {
+    L.q_codes = take(BH * Np * d / 2);
+    L.k_codes = take(BH * Np * d / 2);
+    L.vt_codes = take(BH * d * Np / 2);
+    L.q_scale = take(BH * Np * d / 16);
+    L.k_scale = take(BH * Np * d / 16);
+    L.v_scale = take(BH * d * Np / 16);
+    L.global_scale = take(BH * 3 * sizeof(float));
+  } else {
+    L.q_codes = take(BH * Np * d);
+    L.k_codes = take(BH * Np * d);
+    L.vt_codes = take(BH * d * Np);
+    L.q_scale = take(BH * (Np / 32) * sizeof(float));
+    L.k_scale = take(BH * (Np / 64) * sizeof(float));
+    L.v_scale = take(BH * d * sizeof(float));
+    L.global_scale = take(0);
+  }
+  L.k_mean = take(BH * d * sizeof(float));
+  L.q_mean = take(BH * d * sizeof(float));
+  L.q_bias = take(BH * Np * sizeof(float));
+  // statistics partials [3][BH][Np/64][d] and the V multipliers [BH][d]
+  L.scratch = take((3 * BH * (Np / 64) * d + BH * d) * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+sage::WsPtrs resolve(void* ws, const sage_ws_layout& L) {
+  char* b = (char*)ws;
+  sage::WsPtrs w;
+  w.q_codes = (int8_t*)(b + L.q_codes);
+  w.k_codes = (int8_t*)(b + L.k_codes);
+  w.vt_codes = (uint8_t*)(b + L.vt_codes);
+  w.q_scale = (float*)(b + L.q_scale);
+  w.k_scale = (float*)(b + L.k_scale);
+  w.v_scale = (float*)(b + L.v_scale);
+  w.k_mean = (float*)(b + L.k_mean);
+  w.q_mean = (float*)(b + L.q_mean);
+  w.q_bias = (float*)(b + L.q_bias);
+  w.global_scale = (float*)(b + L.global_scale);
+  w.error = (int*)(b + L.error);
+  w.scratch = (float*)(b + L.scratch);
+  return w;
+}
+
+sage_status check_ws(const void* ws, size_t ws_bytes, const sage_ws_layout& L) {
+  if (!ws) return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null%s");
+  if (((uintptr_t)ws) % kAlign) return set_err(SAGE_ERR_INVALID_ARG, "workspace must be 1024-byte aligned%s");
+  if (ws_bytes < L.total) return set_err(SAGE_ERR_INVALID_ARG, "workspace too small%s");
+  return SAGE_OK;
+}
+
+sage_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SAGE_OK;
+  char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", what, cudaGetErrorString(e));
+  g_last_error = buf;
+  return SAGE_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace sage {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+bool make_tmap_u8_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                     uint32_t box0, uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0, dim0 * dim1};  // bytes, dims 1 and 2
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMapSwizzle sw = box0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace sage
+
+extern "C" {
+
+const char* sage_last_error(void) { return g_last_error.c_str(); }
+
+sage_status sage_workspace_layout(int B, int H, int N, int d, int mode, sage_ws_layout* out) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (!out) return set_err(SAGE_ERR_INVALID_ARG, "layout pointer is null%s");
+  *out = layout_of(B, H, N, d, mode);
+  return SAGE_OK;
+}
+
+size_t sage_workspace_size(int B, int H, int N, int d, int mode) {
+  if (check_shape(B, H, N, d, mode) != SAGE_OK) return 0;
+  return layout_of(B, H, N, d, mode).total;
+}
+
+sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
+                              int smooth_q, int mode, void* ws, size_t ws_bytes, sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (!q || !k || !v) return set_err(SAGE_ERR_INVALID_ARG, "null input pointer%s");
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
+  if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
+    return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
+  if (mode == SAGE_MODE_NVFP4) return set_err(SAGE_ERR_UNSUPPORTED, "NVFP4 mode not built in this library%s");
+  const sage_ws_layout L = layout_of(B, H, N, d, mode);
+  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, 0};
+  const float Vr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 4.5f : 448.0f;
+  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_quant_int8_fp8(q, k, v, pb, Vr, resolve(ws, L), (cudaStream_t)stream),
+                     "quantize launch");
+}
+
+sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
+                                int causal, int smooth_q, int mode, sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (!out) return set_err(SAGE_ERR_INVALID_ARG, "null output pointer%s");
+  if (((uintptr_t)out) % 16) return set_err(SAGE_ERR_INVALID_ARG, "output must be 16-byte aligned%s");
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
+  if (mode != SAGE_MODE_INT8_FP8) return set_err(SAGE_ERR_UNSUPPORTED, "mode not built in this library%s");
+  const sage_ws_layout L = layout_of(B, H, N, d, mode);
+  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
+  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_attn_i8f8(resolve(const_cast<void*>(ws), L), out, pb, 448.0f, (cudaStream_t)stream),
+                     "attention launch");
+}
+
+sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                          int causal, int mode, int dtype, int smooth_q, void* ws, size_t ws_bytes,
+                          sage_stream_t stream) {
+  sage_status st = sage_quantize_qkv(q, k, v, dtype, B, H, N, d, smooth_q, mode, ws, ws_bytes, stream);
+  if (st != SAGE_OK) return st;
+  return sage_attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream);
+}
+
+sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,
+                              int k_tile, int32_t* out, sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, SAGE_MODE_INT8_FP8);
+  if (st != SAGE_OK) return st;
+  const int ntiles = (N + 127) / 128;
+  if (!out || bh < 0 || bh >= B * H || q_tile < 0 || q_tile >= ntiles || k_tile < 0 || k_tile >= ntiles)
+    return set_err(SAGE_ERR_INVALID_ARG, "debug tile out of range%s");
+  const sage_ws_layout L = layout_of(B, H, N, d, SAGE_MODE_INT8_FP8);
+  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  sage::Problem pb{B * H, N, ntiles * 128, d, 0, 0, 0, 0};
+  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_debug_qk(resolve(const_cast<void*>(ws), L), pb, bh, q_tile, k_tile, out,
+                                           (cudaStream_t)stream),
+                     "debug launch");
+}
+
+sage_status sage_debug_timeout_probe(void* ws, size_t ws_bytes, sage_stream_t stream) {
+  if (!ws || ws_bytes < sizeof(int) || ((uintptr_t)ws) % kAlign)
+    return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null or misaligned%s");
+  sage_ws_layout L;
+  memset(&L, 0, sizeof(L));  // only the error word (offset 0) is used
+  sage_status st = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream), "clear");
+  if (st != SAGE_OK) return st;
+  return cuda_status(sage::launch_timeout_probe(resolve(ws, L), (cudaStream_t)stream), "probe launch");
+}
+
+sage_status sage_check(void* ws, size_t ws_bytes, sage_stream_t stream) {
+  if (!ws || ws_bytes < sizeof(int)) return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null%s");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
+  int word = 0;
+  // the error word sits at offset 0 of every layout
+  e = cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e, "error word read");
+  if (word != 0) {
+    const int zero = 0;
+    cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    char buf[64];
+    snprintf(buf, sizeof(buf), "device wait timed out (site 0x%x)", word);
+    g_last_error = buf;
+    return SAGE_ERR_TIMEOUT;
+  }
+  return SAGE_OK;
+}
+
+}  // extern "C"

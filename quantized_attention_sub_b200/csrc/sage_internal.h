@@ -1,0 +1,52 @@
+// sage_internal.h -- declarations shared by the library's translation units
+// (launchers and the resolved workspace pointers).  Not part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sage {
+
+// Device pointers into one workspace, resolved from sage_ws_layout.
+struct WsPtrs {
+  int8_t* q_codes;
+  int8_t* k_codes;
+  uint8_t* vt_codes;
+  float* q_scale;
+  float* k_scale;
+  float* v_scale;
+  float* k_mean;
+  float* q_mean;
+  float* q_bias;
+  float* global_scale;
+  int* error;
+  float* scratch;  // statistics partials, then the per-channel V multipliers
+};
+
+struct Problem {
+  int BH, N, Npad, d, dtype, smooth_q, mode, causal;
+};
+
+// Smoothing statistics + INT8 Q/K + FP8 V (+ bias), enqueued on `s`.
+cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
+                                  const WsPtrs& w, cudaStream_t s);
+
+// Fused attention (FP32 PV accumulator).
+cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s);
+
+// INT32 S tile through the tensor-core path.
+cudaError_t launch_debug_qk(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, int32_t* out,
+                            cudaStream_t s);
+
+// A kernel whose only wait can never complete: exercises the bounded-wait path.
+cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s);
+
+// Tensor maps (cuTensorMapEncodeTiled through the runtime's driver entry point).
+// A 3-D uint8 tensor [dim2][dim1][dim0] with a box of box0 x box1 x 1 and
+// the swizzle that matches a row of box0 bytes (64 or 128).
+bool make_tmap_u8_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                     uint32_t box0, uint32_t box1);
+
+}  // namespace sage

@@ -1,0 +1,78 @@
+"""The C-ABI library loads and exports every symbol include/sage.h declares;
+host-side argument checks and the workspace layout (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_attention_sub_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sage.h")).read()
+    return sorted(set(re.findall(r"SAGE_API\s+[\w\s\*]+?\b(sage_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_attention_sub_b200 import build
+    build.build()
+    return api.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(api.EXPORTED) <= set(names)
+
+
+def test_workspace_layout_is_aligned_and_disjoint(lib):
+    for (B, H, N, d, mode) in [(1, 2, 128, 64, 0), (1, 32, 8192, 128, 0), (1, 12, 32760, 128, 1), (4, 3, 1, 64, 0),
+                               (1, 16, 16384, 128, 2)]:
+        L = api.sage_workspace_layout(B, H, N, d, mode)
+        offs = [getattr(L, f) for f, _ in api.WsLayout._fields_ if f != "total"]
+        assert all(o % 1024 == 0 for o in offs)
+        assert L.total >= max(offs) and api.sage_workspace_size(B, H, N, d, mode) == L.total
+        Np = (N + 127) // 128 * 128
+        if mode != 2:
+            assert L.k_codes - L.q_codes >= B * H * Np * d
+            assert L.vt_codes - L.k_codes >= B * H * Np * d
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 1, 128, 96, 0), api.SAGE_ERR_UNSUPPORTED),
+    ((0, 1, 128, 64, 0), api.SAGE_ERR_INVALID_ARG),
+    ((1, 1, 0, 64, 0), api.SAGE_ERR_INVALID_ARG),
+    ((1, 1, 128, 64, 7), api.SAGE_ERR_INVALID_ARG),
+    ((64, 64, 1 << 20, 128, 0), api.SAGE_ERR_UNSUPPORTED),
+])
+def test_bad_shapes_rejected_on_host(lib, args, status):
+    out = api.WsLayout()
+    assert lib.sage_workspace_layout(*args, ctypes.byref(out)) == status
+    assert api.sage_workspace_size(*args) == 0
+    assert len(lib.sage_last_error()) > 0
+
+
+def test_bad_pointers_rejected_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    ws_bytes = api.sage_workspace_size(1, 2, 128, 64, 0)
+    # null inputs
+    st = lib.sage_quantize_qkv(vp(0), vp(0), vp(0), 0, 1, 2, 128, 64, 0, 0, vp(1024), ws_bytes, vp(0))
+    assert st == api.SAGE_ERR_INVALID_ARG
+    # misaligned workspace
+    st = lib.sage_quantize_qkv(vp(4096), vp(4096), vp(4096), 0, 1, 2, 128, 64, 0, 0, vp(1040), ws_bytes, vp(0))
+    assert st == api.SAGE_ERR_INVALID_ARG
+    # workspace too small
+    st = lib.sage_quantize_qkv(vp(4096), vp(4096), vp(4096), 0, 1, 2, 128, 64, 0, 0, vp(4096), 16, vp(0))
+    assert st == api.SAGE_ERR_INVALID_ARG
+    # bad dtype
+    st = lib.sage_attn_quantized(vp(4096), ws_bytes, vp(4096), 5, 1, 2, 128, 64, 0, 0, 0, vp(0))
+    assert st == api.SAGE_ERR_INVALID_ARG
+    # debug tile out of range
+    st = lib.sage_debug_qk_s32(vp(4096), ws_bytes, 1, 2, 128, 64, 0, 1, 0, vp(4096), vp(0))
+    assert st == api.SAGE_ERR_INVALID_ARG

@@ -1,0 +1,204 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Codes, scales and INT32 QK^T tiles must be bit-exact; the
+output within max-abs 2e-3 and relative-L1 5e-4 of the oracle's."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from quantized_attention_sub_b200 import api, inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L1 = 2e-3, 5e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_attention_sub_b200 import build
+    build.build()
+    api.lib()
+
+
+def run_quant(w, mode, smooth_q, device_inputs=None):
+    q, k, v = device_inputs if device_inputs is not None else [t.cuda() for t in inputs.generate(w)]
+    B, H, N, d = w.shape()
+    ws = api.alloc_workspace(B, H, N, d, mode)
+    api.sage_quantize_qkv(q, k, v, api.DTYPE_CODE[q.dtype], B, H, N, d, smooth_q, mode, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    return (q, k, v), ws, {n: t.cpu().numpy() for n, t in api.ws_views(ws, B, H, N, d, mode).items()}
+
+
+def oracle_quant(qkv, mode, smooth_q):
+    B, H, N, d = qkv[0].shape
+    f = lambda t: t.float().cpu().reshape(B * H, N, d).numpy()
+    return orc.quantize_int8_fp8(f(qkv[0]), f(qkv[1]), f(qkv[2]), smooth_q=smooth_q, mode=mode)
+
+
+def assert_quant_bitexact(g, o, smooth_q):
+    for name in ("q_codes", "k_codes", "vt_codes"):
+        assert np.array_equal(g[name].view(np.uint8), o[name].view(np.uint8)), name
+    for name in ("q_scale", "k_scale", "v_scale", "k_mean"):
+        assert np.array_equal(g[name].view(np.uint32), o[name].view(np.uint32)), name
+    if smooth_q:
+        assert np.array_equal(g["q_mean"].view(np.uint32), o["q_mean"].view(np.uint32))
+        assert np.array_equal(g["q_bias"].view(np.uint32), o["q_bias"].view(np.uint32))
+
+
+SMALL = [
+    # (N, d, dtype, law, smooth_q, mode)
+    (128, 64, "fp16", "k_bias", False, 0),
+    (1, 64, "fp16", "k_bias", False, 0),
+    (31, 128, "bf16", "k_bias_outlier", False, 0),
+    (129, 128, "fp16", "qk_bias", True, 0),
+    (333, 64, "bf16", "qk_bias", True, 1),
+    (1000, 128, "bf16", "k_bias_outlier", False, 0),
+    (700, 128, "fp16", "qk_bias", True, 1),
+]
+
+
+def small_workload(N, d, dtype, law, smooth_q, mode, H=2, causal=False):
+    return inputs.variant(inputs.WORKLOADS["unit"], N=N, d=d, H=H, dtype=dtype, law=law, smooth_q=smooth_q,
+                          mode=mode, causal=causal, seed=5000 + N + d)
+
+
+@pytest.mark.parametrize("N,d,dtype,law,smooth_q,mode", SMALL)
+def test_quantize_bitexact(N, d, dtype, law, smooth_q, mode):
+    w = small_workload(N, d, dtype, law, smooth_q, mode)
+    qkv, ws, g = run_quant(w, mode, smooth_q)
+    assert_quant_bitexact(g, oracle_quant(qkv, mode, smooth_q), smooth_q)
+
+
+def test_quantize_edge_values():
+    """Zero channels, constant tokens, a zero granule, huge and tiny values."""
+    w = small_workload(200, 64, "fp16", "k_bias", True, 0)
+    q, k, v = [t.clone() for t in inputs.generate(w)]
+    v[:, :, :, 5] = 0          # zero V channel -> scale 0, codes 0
+    k[:, :, 64:128, :] = 3.0   # constant K granule -> after smoothing mostly nonzero
+    q[:, 1, 32:64, :] = 0      # zero Q granule when not smoothed
+    v[:, 0, 7, 9] = 60000.0    # big value: other codes of channel 9 go subnormal
+    for smooth_q in (False, True):
+        qkv, ws, g = run_quant(w, 0, smooth_q, [t.cuda() for t in (q, k, v)])
+        o = oracle_quant(qkv, 0, smooth_q)
+        assert_quant_bitexact(g, o, smooth_q)
+    assert np.all(g["vt_codes"][:, 5] == 0) and np.all(g["v_scale"][:, 5] == 0)
+
+
+@pytest.mark.parametrize("N,d", [(128, 64), (333, 128), (1000, 64)])
+def test_qk_s32_tiles_bitexact(N, d):
+    w = small_workload(N, d, "fp16", "k_bias", False, 0)
+    qkv, ws, g = run_quant(w, 0, False)
+    B, H = 1, 2
+    T = (N + 127) // 128
+    out = torch.empty(128, 128, dtype=torch.int32, device="cuda")
+    for bh in range(B * H):
+        for qt, kt in {(0, 0), (T - 1, 0), (0, T - 1), (T - 1, T - 1), (T // 2, (T + 1) // 3)}:
+            api.sage_debug_qk_s32(ws, ws.numel(), B, H, N, d, bh, qt, kt, out)
+            api.sage_check(ws, ws.numel())
+            ref = orc.qk_s32(g["q_codes"][bh, qt * 128:(qt + 1) * 128], g["k_codes"][bh, kt * 128:(kt + 1) * 128])
+            assert np.array_equal(out.cpu().numpy(), ref), (bh, qt, kt)
+
+
+def compare_out(o_gpu, o_ref, dtype, label=""):
+    """Both arrays hold values of `dtype` (the oracle's fp32 result rounded to
+    it).  The max-abs bound 2e-3 applies to every element except rounding
+    flips: two fp32 results straddling a rounding boundary of the output dtype
+    land on adjacent representable values, one ulp apart, and one bf16 ulp of
+    an output above 0.25 in magnitude is already larger than 2e-3.  Flips must
+    stay rare (under 1%) and the relative L1 bound covers every element."""
+    a = o_gpu.astype(np.float64)
+    b = o_ref.astype(np.float64)
+    diff = np.abs(a - b)
+    bits = lambda x: torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(inputs.DTYPES[dtype]).view(
+        torch.int16).numpy().astype(np.int32)
+    adjacent = (np.abs(bits(o_gpu) - bits(o_ref)) == 1) & (np.sign(a) == np.sign(b))
+    bad = (diff > MAX_ABS) & ~adjacent
+    flips = float(np.mean((diff > MAX_ABS) & adjacent))
+    max_abs = float(np.max(np.where(adjacent, 0.0, diff)))
+    rel = float(diff.sum() / max(np.abs(b).sum(), 1e-30))
+    assert not bad.any() and rel <= REL_L1 and flips < 0.01, (label, max_abs, rel, flips)
+    return max_abs, rel, flips
+
+
+def to_dtype_np(x, dtype):
+    return torch.from_numpy(x).to(inputs.DTYPES[dtype]).float().numpy()
+
+
+ATTN_SMALL = [
+    # (N, d, dtype, law, smooth_q, causal)
+    (128, 64, "fp16", "k_bias", False, False),
+    (1, 128, "bf16", "k_bias", False, False),
+    (33, 64, "fp16", "k_bias", False, True),
+    (129, 128, "bf16", "k_bias_outlier", False, True),
+    (333, 128, "fp16", "qk_bias", True, False),
+    (640, 64, "bf16", "qk_bias", True, True),
+    (1000, 128, "bf16", "k_bias_outlier", False, True),
+    (1000, 128, "fp16", "k_bias", False, False),
+]
+
+
+@pytest.mark.parametrize("N,d,dtype,law,smooth_q,causal", ATTN_SMALL)
+def test_attention_matches_oracle(N, d, dtype, law, smooth_q, causal):
+    w = small_workload(N, d, dtype, law, smooth_q, 0, causal=causal)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    B, H = 1, 2
+    ws = api.alloc_workspace(B, H, N, d, 0)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, causal, 0, api.DTYPE_CODE[q.dtype], smooth_q, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    oz = oracle_quant((q, k, v), 0, smooth_q)
+    ref = to_dtype_np(orc.attention_int8_fp8(oz, causal), dtype)
+    got = out.float().cpu().reshape(B * H, N, d).numpy()
+    compare_out(got, ref, dtype, (N, d, dtype, causal))
+
+
+def test_full_size_llm_prefill_sampled_rows():
+    """The B1 H32 N8192 d128 bf16 causal workload at full size, in the launch
+    configuration the bench times: quantization bit-exact everywhere, the
+    output on 24 sampled rows per head (first, last, tile edges, random)."""
+    w = inputs.WORKLOADS["llm_prefill"]
+    B, H, N, d = w.shape()
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    ws = api.alloc_workspace(B, H, N, d, 0)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, True, 0, 1, False, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    g = {n: t.cpu().numpy() for n, t in api.ws_views(ws, B, H, N, d, 0).items()}
+    oz = oracle_quant((q, k, v), 0, False)
+    assert_quant_bitexact(g, oz, False)
+    rng = np.random.default_rng(8192)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 255, 256, N - 129, N - 128, N - 1],
+                                     rng.integers(0, N, 15)])).astype(np.int32)
+    ref = to_dtype_np(orc.attention_int8_fp8(oz, True, rows=rows), "bf16")
+    got = out.float().cpu().reshape(B * H, N, d).numpy()[:, rows]
+    compare_out(got, ref, "bf16", "llm_prefill")
+
+
+def test_repeated_calls_identical_and_no_error():
+    w = small_workload(1000, 128, "bf16", "k_bias", False, 0, causal=True)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    ws = api.alloc_workspace(1, 2, 1000, 128, 0)
+    outs = []
+    for _ in range(3):
+        out = torch.empty_like(q)
+        api.sage_attn_fwd(q, k, v, out, 1, 2, 1000, 128, True, 0, 1, False, ws, ws.numel())
+        outs.append(out)
+    api.sage_check(ws, ws.numel())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    ws = api.alloc_workspace(1, 2, 128, 64, 0)
+    api.sage_debug_timeout_probe(ws, ws.numel())
+    with pytest.raises(api.SageError) as e:
+        api.sage_check(ws, ws.numel())
+    assert e.value.status == api.SAGE_ERR_TIMEOUT
+    # the context still runs work and the word was cleared
+    api.sage_check(ws, ws.numel())
+    w = small_workload(128, 64, "fp16", "k_bias", False, 0)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    out = api.attn_fwd(q, k, v, ws=ws)
+    api.sage_check(ws, ws.numel())
+    assert torch.isfinite(out.float()).all()
