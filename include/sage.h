@@ -104,6 +104,31 @@ SAGE_API size_t sage_workspace_size(int B, int H, int N, int d, int mode);
 SAGE_API sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
                               int smooth_q, int mode, void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* sage_quantize_qkv for callers that cannot allocate device memory.  (The
+ * pages have no counterpart; this is a deployment variant.)  Code running
+ * inside a CUDA-graph capture that must not grow the memory pool, a plugin
+ * whose host framework owns every allocation, or a real-time loop that may
+ * not call the allocator can pass its inputs and one output buffer but no
+ * scratch area.  This entry point keeps the statistics scratch (per-chunk
+ * partial sums) in a 16 MiB device array inside the library instead; every
+ * GPU that loads this part of the library holds that array until the
+ * process exits.  It calls no allocator.
+ *   out: device buffer of at least sage_ws_layout.scratch bytes (everything
+ *        the layout places before `scratch`), 1024-byte aligned; it receives
+ *        the same codes, scales, means and bias as the workspace of
+ *        sage_quantize_qkv, at the same offsets.
+ *   Limit: 3*B*H*(Npad/64)*d + B*H*d floats <= 4 Mi (16 MiB); larger problems
+ *   return SAGE_ERR_UNSUPPORTED with the sizes in sage_last_error().
+ *   The first call on a device looks up the array's device address once,
+ *   with that device current; make that first call before any stream
+ *   capture.  All calls share the array: calls that overlap on the GPU (on
+ *   different streams, or on several host threads at once) race on it and
+ *   must be serialized by the caller.  Nothing in the array needs to start at
+ *   zero; each call overwrites what it reads. */
+SAGE_API sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v, int dtype, int B, int H,
+                                              int N, int d, int smooth_q, int mode, void* out, size_t out_bytes,
+                                              sage_stream_t stream);
+
 /* Fused attention on a workspace filled by sage_quantize_qkv with the same
  * (B,H,N,d,smooth_q,mode): per 128-query tile, for each 128-key tile, INT8
  * QK^T on the tensor cores, dequantize (scale_q * scale_k, plus the Q bias),

@@ -19,7 +19,8 @@ SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_CUDA, SAGE_ERR_TIM
 MODE_INT8_FP8, MODE_INT8_FP8_F16ACC, MODE_NVFP4 = 0, 1, 2
 DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
 
-EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_attn_quantized",
+EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_quantize_qkv_static",
+            "sage_attn_quantized",
             "sage_attn_fwd", "sage_debug_qk_s32", "sage_debug_timeout_probe", "sage_check", "sage_last_error")
 
 
@@ -53,6 +54,8 @@ def lib() -> ctypes.CDLL:
         L.sage_workspace_size.restype = sz
         L.sage_quantize_qkv.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
         L.sage_quantize_qkv.restype = i
+        L.sage_quantize_qkv_static.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_quantize_qkv_static.restype = i
         L.sage_attn_quantized.argtypes = [vp, sz, vp, i, i, i, i, i, i, i, i, vp]
         L.sage_attn_quantized.restype = i
         L.sage_attn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
@@ -97,6 +100,14 @@ def sage_workspace_size(B, H, N, d, mode) -> int:
 def sage_quantize_qkv(q, k, v, dtype, B, H, N, d, smooth_q, mode, ws, ws_bytes, stream=None):
     _raise(lib().sage_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), dtype, B, H, N, d, int(smooth_q), mode, _ptr(ws),
                                    ws_bytes, _stream(stream)))
+
+
+def sage_quantize_qkv_static(q, k, v, dtype, B, H, N, d, smooth_q, mode, out, out_bytes, stream=None):
+    """No-allocation quantization (see include/sage.h): `out` receives the
+    quantized region of the workspace layout; the statistics scratch lives in
+    a fixed 16 MiB device array inside the library."""
+    _raise(lib().sage_quantize_qkv_static(_ptr(q), _ptr(k), _ptr(v), dtype, B, H, N, d, int(smooth_q), mode,
+                                          _ptr(out), out_bytes, _stream(stream)))
 
 
 def sage_attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream=None):

@@ -177,6 +177,38 @@ sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int d
                      "quantize launch");
 }
 
+sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v, int dtype, int B, int H, int N,
+                                     int d, int smooth_q, int mode, void* out, size_t out_bytes,
+                                     sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (!q || !k || !v) return set_err(SAGE_ERR_INVALID_ARG, "null input pointer%s");
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
+  if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
+    return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
+  if (mode == SAGE_MODE_NVFP4) return set_err(SAGE_ERR_UNSUPPORTED, "NVFP4 mode not built in this library%s");
+  if (!out) return set_err(SAGE_ERR_INVALID_ARG, "output buffer pointer is null%s");
+  if (((uintptr_t)out) % kAlign) return set_err(SAGE_ERR_INVALID_ARG, "output buffer must be 1024-byte aligned%s");
+  const sage_ws_layout L = layout_of(B, H, N, d, mode);
+  if (out_bytes < L.scratch)
+    return set_err(SAGE_ERR_INVALID_ARG, "output buffer smaller than the layout's quantized region (layout.scratch)%s");
+  const size_t Np = ((size_t)N + 127) / 128 * 128, BH = (size_t)B * H;
+  const size_t need = 3 * BH * (Np / 64) * d + BH * d;
+  if (need > sage::static_scratch_floats()) {
+    char buf[200];
+    snprintf(buf, sizeof(buf), "problem needs %zu floats of static scratch; the maximum is %zu (16 MiB)", need,
+             sage::static_scratch_floats());
+    g_last_error = buf;
+    return SAGE_ERR_UNSUPPORTED;
+  }
+  sage::Problem pb{B * H, N, (int)Np, d, dtype, smooth_q ? 1 : 0, mode, 0};
+  const float Vr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 4.5f : 448.0f;
+  if ((st = cuda_status(cudaMemsetAsync((char*)out + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_quant_static(q, k, v, pb, Vr, resolve(out, L), (cudaStream_t)stream),
+                     "static quantize launch");
+}
+
 sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
                                 int causal, int smooth_q, int mode, sage_stream_t stream) {
   sage_status st = check_shape(B, H, N, d, mode);

@@ -33,6 +33,12 @@ struct Problem {
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
                                   const WsPtrs& w, cudaStream_t s);
 
+// The same quantization pass with its statistics scratch in a file-scope
+// device array (quant_static.cu) instead of w.scratch, which is ignored.
+cudaError_t launch_quant_static(const void* q, const void* k, const void* v, const Problem& pb, float Vr, WsPtrs w,
+                                cudaStream_t s);
+size_t static_scratch_floats();
+
 // Fused attention (FP32 PV accumulator).
 cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s);
 
