@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.orc_f16_round.restype = ctypes.c_double
         L.orc_f16_round.argtypes = [ctypes.c_double]
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_exp2.restype = ctypes.c_float
+        L.orc_exp2.argtypes = [ctypes.c_float]
     return _lib
 
 
@@ -113,6 +115,11 @@ def e2m1_decode(c: int) -> float:
 
 def f16_round(x: float) -> float:
     return lib().orc_f16_round(float(x))
+
+
+def exp2(d: float) -> float:
+    """The exp2 both sides use (range reduction + degree-4 polynomial)."""
+    return lib().orc_exp2(float(d))
 
 
 def e4m3_decode_array(codes: np.ndarray) -> np.ndarray:

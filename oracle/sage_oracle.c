@@ -153,6 +153,34 @@ ORC_EXPORT double orc_f16_round(double x)
   return x < 0 ? -r : r;
 }
 
+/* exp2 as both sides compute it.  The pages fix no accuracy for the softmax
+ * exponential; this reading fixes one, so that the FP8 decision P~ =
+ * e4m3(2^d) is the same bit for bit on the CPU and on the GPU.  Method:
+ * Cody-Waite style range reduction d = n + f (n = floor(d), f in [0,1), both
+ * exact in fp32), a degree-3 polynomial for 2^f with its constant term fixed
+ * to 1 (coefficients from a Remez exchange on the relative error; max relative
+ * error 8.6e-5 in fp32 Horner form, far below the 2^-4 step of e4m3; exact at
+ * integers, so a row max that does not move gives alpha = 1), then n added to
+ * the exponent field.  d is clamped to -127 first (NaN included), where the
+ * result is +0. */
+static const float EXP2_C1 = 0x1.63e658p-1f;
+static const float EXP2_C2 = 0x1.d2378ap-3f;
+static const float EXP2_C3 = 0x1.3baaa6p-4f;
+
+ORC_EXPORT float orc_exp2(float d)
+{
+  if (!(d > -127.0f)) d = -127.0f;
+  float n = floorf(d);
+  float f = d - n;
+  float r = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.0f);
+  uint32_t rb;
+  memcpy(&rb, &r, 4);
+  rb += ((uint32_t)(int32_t)n) << 23;
+  float out;
+  memcpy(&out, &rb, 4);
+  return out;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Smoothing statistics (SageAttention2 abstract: smoothing; the mean is over */
 /* tokens, per channel).                                                      */
@@ -313,57 +341,65 @@ enum { ORC_MODE_FP32ACC = 0, ORC_MODE_F16ACC = 1 };
 
 /* One query row, FlashAttention order: key tiles of 128 in ascending order.
  * Per tile (only tiles holding at least one key the row may see):
- *   t_j   = (float(S_ij) * (sq_i * sk_g(j)) + bias_j) * (log2(e) / sqrt(d))
- *   m_new = max(m, max_j t_j);  alpha = exp2(m - m_new)
- *   p_j   = exp2(t_j - m_new);  l = alpha * l + sum_j p_j  (p before rounding)
- *   p~_j  = e4m3(p_j * Pr)
- *   FP32 accumulator: acc_c = alpha * acc_c + fl32(exact sum_j p~_j v^_jc)
+ *   kf    = (sq_i * sk_g(j)) * (log2(e) / sqrt(d))        one factor per 64-key granule
+ *   t_j   = float(S_ij) * kf, or fma(float(S_ij), kf, bias_j * (log2(e)/sqrt(d)))
+ *   m_new = max(m, max_j t_j);  alpha = exp2(m - m_new);  m' = m_new - log2(Pr)
+ *   p'_j  = exp2(d_j) with d_j = fma(float(S_ij), kf, -m') (no bias) or t_j - m'
+ *           -- p'_j = p_j * Pr with p_j the softmax numerator;
+ *   l     = alpha * l + sum_j p'_j        (in units of Pr)
+ *   P~_j  = e4m3(p'_j)
+ *   FP32 accumulator: acc_c = alpha * acc_c + fl32(exact sum_j P~_j v^_jc)
  *   FP16 accumulator (SageAttention2++ Sec. 3.2): per 64-key chunk,
  *        h = f16(exact sum of its first 32 products), h = f16(h + exact sum of
  *        the next 32); acc_c = alpha * acc_c + h_chunk0 + h_chunk1
- *   O_ic  = acc_c * scale_v[c] / (Pr * l)
- * Masked keys (j >= N, or j > i when causal) take no part.  The exact sums of
- * e4m3 products fit a double: each product has 8 significant bits within
- * 2^-18..2^18 and at most 128 are added.
+ *   O_ic  = acc_c * scale_v[c] / l
+ * exp2 is orc_exp2 above.  Masked keys (j >= N, or j > i when causal) take no
+ * part.  The exact sums of e4m3 products fit a double: each product has 8
+ * significant bits within 2^-18..2^18 and at most 128 are added.
  * out_row receives fp32 results (the caller rounds to the output dtype). */
 static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* vt,
                      float sq, const float* sk, const float* bias, const float* scale_v,
                      int N, int Npad, int d, int causal, int mode, float Pr,
-                     float* acc, float* tvals, float* pvals, int* pcode, float* out_row)
+                     float* acc, float* tvals, float* xvals, int* pcode, float* out_row)
 {
   const float c_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+  const float log2Pr = (float)log2((double)Pr);
   float m = -INFINITY, l = 0.0f;
   for (int c = 0; c < d; ++c) acc[c] = 0.0f;
   int jmax = causal ? (i < N - 1 ? i : N - 1) : N - 1;   /* last visible key */
   for (int j0 = 0; j0 <= jmax; j0 += 128) {
-    int j1 = j0 + 128;                                  /* tile [j0, j1) */
     float mt = -INFINITY;
-    for (int j = j0; j < j1; ++j) {
+    for (int j = j0; j < j0 + 128; ++j) {
       if (j > jmax) { tvals[j - j0] = -INFINITY; continue; }
       int32_t s = 0;
       for (int c = 0; c < d; ++c) s += (int32_t)qc[(size_t)i * d + c] * (int32_t)kc[(size_t)j * d + c];
-      float t = (float)s * (sq * sk[j / 64]);
-      if (bias) t = t + bias[j];
-      t = t * c_log2;
+      const float x = (float)s;
+      const float kf = (sq * sk[j / 64]) * c_log2;
+      const float t = bias ? fmaf(x, kf, bias[j] * c_log2) : x * kf;
+      xvals[j - j0] = x;
       tvals[j - j0] = t;
       if (t > mt) mt = t;
     }
-    float m_new = m > mt ? m : mt;
-    float alpha = exp2f(m - m_new);          /* m = -inf on the first tile: 0 */
+    const float m_new = m > mt ? m : mt;
+    const float alpha = orc_exp2(m - m_new);   /* first tile: exp2(-inf) = 0 */
+    const float mp = m_new - log2Pr;
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
-      float p = (j0 + j > jmax) ? 0.0f : exp2f(tvals[j] - m_new);
-      pvals[j] = p;
+      float p = 0.0f;
+      if (j0 + j <= jmax) {
+        const float kf = (sq * sk[(j0 + j) / 64]) * c_log2;
+        const float dj = bias ? tvals[j] - mp : fmaf(xvals[j], kf, -mp);
+        p = orc_exp2(dj);
+      }
       ps = ps + p;
-      pcode[j] = orc_e4m3_encode((double)(p * Pr));
+      pcode[j] = orc_e4m3_encode((double)p);
     }
     l = alpha * l + ps;
     for (int c = 0; c < d; ++c) {
       const uint8_t* vrow = vt + (size_t)c * Npad + j0;
       if (mode == ORC_MODE_FP32ACC) {
         double sum = 0.0;
-        for (int j = 0; j < 128; ++j)
-          if (j0 + j < Npad) sum += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
+        for (int j = 0; j < 128; ++j) sum += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
         acc[c] = alpha * acc[c] + (float)sum;
       } else {
         float a = alpha * acc[c];
@@ -380,8 +416,7 @@ static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* v
     }
     m = m_new;
   }
-  float denom = Pr * l;
-  for (int c = 0; c < d; ++c) out_row[c] = acc[c] * scale_v[c] / denom;
+  for (int c = 0; c < d; ++c) out_row[c] = acc[c] * scale_v[c] / l;
 }
 
 /* Attention output for the listed query rows of every (b,h) slice.
@@ -397,7 +432,7 @@ ORC_EXPORT void orc_attn_int8_fp8(const int8_t* qc, const float* sq, const int8_
   {
     float* acc = (float*)malloc(sizeof(float) * d);
     float* tv = (float*)malloc(sizeof(float) * 128);
-    float* pv = (float*)malloc(sizeof(float) * 128);
+    float* xv = (float*)malloc(sizeof(float) * 128);
     int* pc = (int*)malloc(sizeof(int) * 128);
 #pragma omp for schedule(dynamic, 4) collapse(2)
     for (int bh = 0; bh < BH; ++bh)
@@ -406,10 +441,10 @@ ORC_EXPORT void orc_attn_int8_fp8(const int8_t* qc, const float* sq, const int8_
         attn_row(i, qc + (size_t)bh * Npad * d, kc + (size_t)bh * Npad * d,
                  vt + (size_t)bh * d * Npad, sq[(size_t)bh * (Npad / 32) + i / 32],
                  sk + (size_t)bh * (Npad / 64), bias ? bias + (size_t)bh * Npad : NULL,
-                 scale_v + (size_t)bh * d, N, Npad, d, causal, mode, Pr, acc, tv, pv, pc,
+                 scale_v + (size_t)bh * d, N, Npad, d, causal, mode, Pr, acc, tv, xv, pc,
                  out + ((size_t)bh * nrows + r) * d);
       }
-    free(acc); free(tv); free(pv); free(pc);
+    free(acc); free(tv); free(xv); free(pc);
   }
 }
 
@@ -528,10 +563,10 @@ static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq
       if (t > mt) mt = t;
     }
     float m_new = m > mt ? m : mt;
-    float alpha = exp2f(m - m_new);
+    float alpha = orc_exp2(m - m_new);
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
-      float p = (j0 + j > jmax) ? 0.0f : exp2f(tvals[j] - m_new);
+      float p = (j0 + j > jmax) ? 0.0f : orc_exp2(tvals[j] - m_new);
       pvals[j] = p;
       ps = ps + p;
     }

@@ -4,23 +4,27 @@
 // V scale, rescale at the end).
 //
 // One CTA owns two 128-query tiles of one (b, h) slice and walks the key
-// tiles of 128 in order.  Warp roles (384 threads):
-//   warps 0-3  softmax warpgroup of query tile 0 (thread r <-> row r <-> TMEM lane r)
-//   warps 4-7  softmax warpgroup of query tile 1
-//   warp  8    TMA producer (Q tiles once, then a 3-stage ring of K and V^T tiles);
-//              also owns the TMEM allocation
-//   warp  9    MMA issuer (one thread): S_q = Q_q K^T with tcgen05 kind::i8 into
-//              TMEM, O_q += P~_q V with kind::f8f6f4 into TMEM
-//   warps 10-11 idle
+// tiles of 128 in order.  Warp roles (576 threads, 18 warps):
+//   warps 0-15  softmax: warpgroup g = warp / 4 handles query tile q = g / 2
+//               and key half h = g % 2 (keys [64h, 64h + 64) of every tile,
+//               one 64-key scale granule); thread <-> row <-> TMEM lane.
+//               Each SM sub-partition runs one warp of every warpgroup.
+//   warp 16     TMA producer (Q tiles once, then a 3-stage ring of K and V^T
+//               tiles); owns the TMEM allocation
+//   warp 17     MMA issuer (one thread): S_q = Q_q K^T with tcgen05 kind::i8
+//               into TMEM, O_q += P~_q V with kind::f8f6f4 into TMEM
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 after it.
-// Per key tile j the softmax thread of row i:
-//   loads S(i, j-tile) from TMEM and frees the S buffer,
-//   t = (float(S) * (sq_i * sk_g) + bias_j) * log2(e)/sqrt(d), masked keys -inf,
-//   m_new = max(m, max t), alpha = exp2(m - m_new),
-//   waits for the previous P~V, multiplies its O row by alpha (skipped when
-//   alpha == 1 on the whole warp), writes P~ = e4m3(exp2(t - m_new) * Pr) into
-//   the 128B-swizzled K-major shared tile the MMA reads, l = alpha l + sum p.
-// At the end O = acc * scale_v / (Pr * l) is cast and stored.
+// Per key tile j the two threads of row i (one per key half):
+//   load their 64 S values from TMEM and free the S buffer,
+//   take the half's logit max and exchange it through shared memory,
+//   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
+//   p' = exp2(d) with d = t - m_new + log2(Pr), P~ = e4m3(p'),
+//   wait for the previous P~V, multiply their half of the O row by alpha
+//   (skipped when alpha == 1 on the whole warp), write their 64 P~ bytes into
+//   the 128B-swizzled K-major shared tile the MMA reads, l_h = alpha l_h + sum p'.
+// At the end l = l_0 + l_1 and O = acc * scale_v / l is cast and stored.
+// exp2 is the method's own (range reduction + degree-3 polynomial), so the P~
+// codes equal those of the CPU reference computation bit for bit.
 // Every wait is bounded (sage_ptx.cuh); a timeout records an error code in
 // the workspace, makes the other roles stop, and the CTA frees its TMEM.
 #include <cuda_bf16.h>
@@ -34,7 +38,9 @@ namespace sage {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kThreads = 384;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16, kMmaWarp = 17;
+constexpr int kThreads = 32 * 18;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -48,7 +54,10 @@ struct Smem {
   static constexpr int off_v = off_k + kStages * kK;
   static constexpr int off_p = off_v + kStages * kV;
   static constexpr int off_bar = off_p + 2 * kP;
-  static constexpr int bytes = off_bar + 256;
+  // row-max / row-sum exchange between the two key halves:
+  // [query tile 2][tile parity 2][half 2][row 128] floats
+  static constexpr int off_x = off_bar + 256;
+  static constexpr int bytes = off_x + 2 * 2 * 2 * 128 * 4;
   static constexpr int alloc = bytes + 1024;  // room to align the base to 1024
 };
 
@@ -60,7 +69,7 @@ struct AttnArgs {
   void* out;
   int* err;
   int N, Npad, causal, num_pairs;
-  float c_log2, Pr;
+  float c_log2, log2Pr;
 };
 
 // error codes: 0x100 | site
@@ -75,6 +84,49 @@ enum : int {
 SAGE_DEV void fail(volatile int* abort_flag, int* err, int code) {
   *abort_flag = 1;
   atomicCAS(err, 0, code);
+}
+
+// 1.5 * 2^23: for |S| < 2^22 the bits (S + kMagicI) read as a float equal
+// kMagicF + S exactly (|S| <= 128 * 127^2 < 2^21 here).
+constexpr uint32_t kMagicI = 0x4B400000u;
+constexpr float kMagicF = 12582912.0f;
+
+SAGE_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2 of the method, the same definition the CPU reference computation uses:
+// d clamped to -127 (NaN included), d = n + f with n = floor(d) (the
+// round-down add of 1.5*2^23 gives 1.5*2^23 + n exactly), 2^f by a degree-3
+// polynomial with constant term 1 (Remez fit of the relative error, max
+// 8.6e-5), then n added to the exponent field.  2^(integer) is exact; d <= -127
+// gives +0.
+constexpr float kE1 = 0x1.63e658p-1f, kE2 = 0x1.d2378ap-3f, kE3 = 0x1.3baaa6p-4f;
+
+SAGE_DEV float exp2m(float d) {
+  d = fmaxf(d, -127.0f);
+  const float y = __fadd_rd(d, kMagicF);
+  const float f = __fadd_rn(d, -__fadd_rn(y, -kMagicF));
+  float r = __fmaf_rn(kE3, f, kE2);
+  r = __fmaf_rn(r, f, kE1);
+  r = __fmaf_rn(r, f, 1.0f);
+  return __uint_as_float(__float_as_uint(r) + (__float_as_uint(y) << 23));
+}
+
+// The same on a pair, with the packed f32x2 ALU operations.
+SAGE_DEV float2 exp2m2(float2 d) {
+  d.x = fmaxf(d.x, -127.0f);
+  d.y = fmaxf(d.y, -127.0f);
+  const float2 y = __fadd2_rd(d, make_float2(kMagicF, kMagicF));
+  const float2 n = __fadd2_rn(y, make_float2(-kMagicF, -kMagicF));
+  const float2 f = __fadd2_rn(d, make_float2(-n.x, -n.y));
+  float2 r = __ffma2_rn(make_float2(kE3, kE3), f, make_float2(kE2, kE2));
+  r = __ffma2_rn(r, f, make_float2(kE1, kE1));
+  r = __ffma2_rn(r, f, make_float2(1.0f, 1.0f));
+  return make_float2(__uint_as_float(__float_as_uint(r.x) + (__float_as_uint(y.x) << 23)),
+                     __uint_as_float(__float_as_uint(r.y) + (__float_as_uint(y.y) << 23)));
 }
 
 SAGE_DEV float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -95,11 +147,12 @@ SAGE_DEV uint32_t pack2<__nv_bfloat16>(float a, float b) {
 
 }  // namespace
 
-template <int D, typename OutT>
+template <int D, typename OutT, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using L = Smem<D>;
+  constexpr int kHalfD = D / 2;  // O columns each key half rescales and stores
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(smem + L::off_bar);
@@ -108,13 +161,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = bars + 1 + kStages;
   uint64_t* v_full = bars + 1 + 2 * kStages;
   uint64_t* v_empty = bars + 1 + 3 * kStages;
-  uint64_t* s_full = bars + 1 + 4 * kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* o_done = s_full + 6;
-  uint64_t* mma_fin = s_full + 8;
-  uint32_t* tmem_slot = (uint32_t*)(s_full + 9);
+  uint64_t* s_full = bars + 1 + 4 * kStages;  // [2]
+  uint64_t* s_free = s_full + 2;              // [2]
+  uint64_t* p_full = s_full + 4;              // [2]
+  uint64_t* o_done = s_full + 6;              // [2]
+  uint64_t* x_bar = s_full + 8;               // [2 query tiles][2 parities]
+  uint64_t* mma_fin = s_full + 12;
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 13);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* xch = (float*)(smem + L::off_x);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = a.causal ? (a.num_pairs - 1 - (int)blockIdx.x) : (int)blockIdx.x;
@@ -138,15 +193,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&s_full[q], 1);
-      mbar_init(&s_free[q], 4);
-      mbar_init(&p_full[q], 4);
+      mbar_init(&s_free[q], 8);   // 8 softmax warps per query tile
+      mbar_init(&p_full[q], 8);
       mbar_init(&o_done[q], 1);
+      mbar_init(&x_bar[2 * q], 256);
+      mbar_init(&x_bar[2 * q + 1], 256);
     }
     mbar_init(mma_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -155,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -191,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
         if (!mbar_wait(&v_full[j % kStages], (j / kStages) & 1, &no_abort)) atomicCAS(a.err, 0, kErrDrain);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_make(2u, 1u, 1u, 128, 128);  // s32 <- s8 x s8
@@ -226,15 +283,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (next_k) {
           const int s1 = (j + 1) % kStages;
           if (!(ok = mbar_wait(&k_full[s1], ((j + 1) / kStages) & 1, abort_flag))) break;
+          tc_fence_after();
         }
-        if (!(ok = mbar_wait(&v_full[j % kStages], (j / kStages) & 1, abort_flag))) break;
-        tc_fence_after();
+        // next S tiles first (they need only the S buffers back), then P~V
         for (int q = 0; q < 2 && ok; ++q) {
           if (j + 1 < nt[q]) {
             if (!(ok = mbar_wait(&s_free[q], j & 1, abort_flag))) break;
             tc_fence_after();
             issue_s(q, j + 1);
           }
+        }
+        if (!ok) break;
+        if (next_k) tc_commit(&k_empty[(j + 1) % kStages]);
+        if (!(ok = mbar_wait(&v_full[j % kStages], (j / kStages) & 1, abort_flag))) break;
+        tc_fence_after();
+        for (int q = 0; q < 2 && ok; ++q) {
           if (j < nt[q]) {
             if (!(ok = mbar_wait(&p_full[q], j & 1, abort_flag))) break;
             tc_fence_after();
@@ -242,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        if (next_k) tc_commit(&k_empty[(j + 1) % kStages]);
         tc_commit(&v_empty[j % kStages]);
       }
       if (!ok) fail(abort_flag, a.err, kErrMma);
@@ -251,9 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int no_abort = 0;
       if (!mbar_wait(mma_fin, 0, &no_abort)) atomicCAS(a.err, 0, kErrDrain);
     }
-  } else if (warp < 8) {
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
-    const int q = warp >> 2;
+    const int g = warp >> 2;          // warpgroup
+    const int q = g >> 1, h = g & 1;  // query tile, key half
     const int r = threadIdx.x & 127;
     const int w4 = warp & 3;
     if (nt[q] > 0) {
@@ -261,11 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = qt * 128 + r;
       const float sq = a.q_scale[(size_t)bh * (a.Npad / 32) + (row >> 5)];
       const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
-      const uint32_t t_s = tmem + lane_off + q * 128;
-      const uint32_t t_o = tmem + lane_off + 256 + q * D;
+      const uint32_t t_s = tmem + lane_off + q * 128 + h * 64;
+      const uint32_t t_o = tmem + lane_off + 256 + q * D + h * kHalfD;
       uint8_t* prow = smem + L::off_p + q * L::kP + r * 128;
       const float* ksc = a.k_scale + (size_t)bh * (a.Npad / 64);
-      const float* brow = a.bias ? a.bias + (size_t)bh * a.Npad : nullptr;
+      const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
+      float* xq = xch + q * 512;  // [parity][half][row]
+      // m: running row max of the logits (log2 units); l: this half's running
+      // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nt[q]; ++j) {
@@ -275,32 +341,106 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[128];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_ld32(t_s + 32 * i, sr + 32 * i);
+        uint32_t sr[64];
+        tmem_ld32(t_s, sr);
+        tmem_ld32(t_s + 32, sr + 32);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
 
-        const float f0 = __fmul_rn(sq, ksc[2 * j]), f1 = __fmul_rn(sq, ksc[2 * j + 1]);
-        const int kbase = j * 128;
-        const bool need_mask = (kbase + 127 >= a.N) || (a.causal && j == qt);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float t = __fmul_rn((float)(int)sr[c], c < 64 ? f0 : f1);
-          if (brow) t = __fadd_rn(t, __ldg(brow + kbase + c));
-          t = __fmul_rn(t, a.c_log2);
-          if (need_mask) {
-            const int kj = kbase + c;
-            if (kj >= a.N || (a.causal && kj > row)) t = -INFINITY;
-          }
-          sr[c] = f2u(t);
-          mx = fmaxf(mx, t);
+        // Logits and P~ follow the method's fp32 steps exactly (the CPU
+        // reference computation takes the same ones):
+        //   kf = (sq * sk) * log2(e)/sqrt(d) for this half's 64-key granule,
+        //   t  = float(S) * kf  (or fma(float(S), kf, bias * log2(e)/sqrt(d))),
+        //   m' = max - log2(Pr),  d = fma(float(S), kf, -m')  (or t - m'),
+        //   p' = exp2m(d) = p * Pr,  P~ = e4m3(p').
+        const float kf = __fmul_rn(__fmul_rn(sq, ksc[2 * j + h]), a.c_log2);
+        const int kbase = j * 128 + h * 64;
+        // visible keys of this row among the half's 64 form the prefix c < lim
+        int lim = 64;
+        if (kbase + 63 >= a.N || (a.causal && j == qt)) {
+          lim = min(lim, a.N - kbase);
+          if (a.causal) lim = min(lim, row - kbase + 1);
         }
-        const float m_new = fmaxf(m, mx);
-        const float alpha = exp2f(m - m_new);
+        // S + 1.5*2^23 read as a float is exactly 1.5*2^23 + S (|S| < 2^22),
+        // and positive floats order like their integers.  Masked keys become
+        // -inf: below every biased value in the max, and d = -inf (or NaN
+        // for a zero scale) clamps to -127, where exp2m gives +0.
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sr[c] += kMagicI;
+        if (lim < 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c >= lim) sr[c] = 0xFF800000u;
+        }
+        const float2 nmag = make_float2(-kMagicF, -kMagicF);
+        float mt;
+        if (!HAS_BIAS) {
+          float ga = -INFINITY, gb = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            ga = fmax3(ga, u2f(sr[c]), u2f(sr[c + 1]));
+            gb = fmax3(gb, u2f(sr[c + 2]), u2f(sr[c + 3]));
+          }
+          // a half with no visible key gives -inf, or NaN for a zero scale
+          mt = __fmul_rn(fmaxf(ga, gb) - kMagicF, kf);
+        } else {
+          const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
+          const float2 cl2 = make_float2(a.c_log2, a.c_log2);
+          float ma = -INFINITY, mb = -INFINITY;
+#pragma unroll
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 bv = __ldg(b4 + c4);
+            const int c = 4 * c4;
+            const float2 xa = __fadd2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), nmag);
+            const float2 xb = __fadd2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), nmag);
+            const float2 ta = __ffma2_rn(xa, make_float2(kf, kf), __fmul2_rn(make_float2(bv.x, bv.y), cl2));
+            const float2 tb = __ffma2_rn(xb, make_float2(kf, kf), __fmul2_rn(make_float2(bv.z, bv.w), cl2));
+            sr[c] = f2u(ta.x);
+            sr[c + 1] = f2u(ta.y);
+            sr[c + 2] = f2u(tb.x);
+            sr[c + 3] = f2u(tb.y);
+            // masked keys carry -inf (or NaN for a zero scale): fmax3 ignores NaN
+            ma = fmax3(ma, ta.x, ta.y);
+            mb = fmax3(mb, tb.x, tb.y);
+          }
+          mt = fmaxf(ma, mb);
+        }
+        // exchange the half maxima of the row (slot parity alternates per tile)
+        float* xs = xq + (j & 1) * 256;
+        xs[h * 128 + r] = mt;
+        mbar_arrive(&x_bar[2 * q + (j & 1)]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&x_bar[2 * q + (j & 1)], (j >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        mt = fmaxf(mt, xs[(h ^ 1) * 128 + r]);
+        const float m_new = fmaxf(m, mt);
+        const float alpha = exp2m(m - m_new);  // +0 on the first tile (m = -inf), 1 if the max stays
+        const float mp = m_new - a.log2Pr;
+
+        // p' = p * Pr for the 64 keys, P~ = e4m3(p') packed 4 per word, and
+        // the sum of p'
+        uint32_t pw[16];
+        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+        const float2 nmp = make_float2(-mp, -mp), kf2 = make_float2(kf, kf);
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const int c = 4 * c4;
+          float2 da, db;
+          if (!HAS_BIAS) {
+            da = __ffma2_rn(__fadd2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), nmag), kf2, nmp);
+            db = __ffma2_rn(__fadd2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), nmag), kf2, nmp);
+          } else {
+            da = __fadd2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), nmp);
+            db = __fadd2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), nmp);
+          }
+          const float2 pa = exp2m2(da), pb = exp2m2(db);
+          sa = __fadd2_rn(sa, pa);
+          sb = __fadd2_rn(sb, pb);
+          pw[c4] = (uint32_t)e4m3x2(pa.x, pa.y) | ((uint32_t)e4m3x2(pb.x, pb.y) << 16);
+        }
         if (j > 0) {
           // P~V of the previous tile must be done: its P buffer is reused and
           // its O rows are rescaled below.
@@ -311,65 +451,65 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-            for (int i = 0; i < D / 32; ++i) {
+            for (int i = 0; i < kHalfD / 32; ++i) {
               uint32_t o[32];
               tmem_ld32(t_o + 32 * i, o);
               tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = f2u(__fmul_rn(u2f(o[e]), alpha));
+              for (int e = 0; e < 32; e += 2) {
+                const float2 v2 = __fmul2_rn(make_float2(u2f(o[e]), u2f(o[e + 1])), make_float2(alpha, alpha));
+                o[e] = f2u(v2.x);
+                o[e + 1] = f2u(v2.y);
+              }
               tmem_st32(t_o + 32 * i, o);
             }
             tmem_st_wait();
           }
         }
-        float ps = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k0 = cc * 16 + e * 4;
-            const float p0 = exp2f(u2f(sr[k0]) - m_new), p1 = exp2f(u2f(sr[k0 + 1]) - m_new);
-            const float p2 = exp2f(u2f(sr[k0 + 2]) - m_new), p3 = exp2f(u2f(sr[k0 + 3]) - m_new);
-            ps = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(ps, p0), p1), p2), p3);
-            const uint32_t lo = e4m3x2(__fmul_rn(p0, a.Pr), __fmul_rn(p1, a.Pr));
-            const uint32_t hi = e4m3x2(__fmul_rn(p2, a.Pr), __fmul_rn(p3, a.Pr));
-            w[e] = lo | (hi << 16);
-          }
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        for (int cc = 0; cc < 4; ++cc)
+          *reinterpret_cast<uint4*>(prow + (((4 * h + cc) ^ (r & 7)) << 4)) =
+              make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[q]);
-        l = __fadd_rn(__fmul_rn(alpha, l), ps);
+        l = __fadd_rn(__fmul_rn(alpha, l), (sa.x + sa.y) + (sb.x + sb.y));
         m = m_new;
       }
       if (ok && !__all_sync(0xffffffffu, mbar_wait(&o_done[q], (nt[q] - 1) & 1, abort_flag))) ok = false;
+      if (ok) {
+        // the row sum is the sum of both halves' sums
+        const int jx = nt[q];
+        float* xs = xq + (jx & 1) * 256;
+        xs[h * 128 + r] = l;
+        mbar_arrive(&x_bar[2 * q + (jx & 1)]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&x_bar[2 * q + (jx & 1)], (jx >> 1) & 1, abort_flag))) ok = false;
+        else l = h == 0 ? __fadd_rn(l, xs[128 + r]) : __fadd_rn(xs[r], l);
+      }
       if (!ok) {
         fail(abort_flag, a.err, kErrSoftmax);
       } else {
         tc_fence_after();
-        const float inv = __frcp_rn(__fmul_rn(a.Pr, l));
-        const float* vs = a.v_scale + (size_t)bh * D;
-        OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D;
+        const float* vs = a.v_scale + (size_t)bh * D + h * kHalfD;
+        OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D + h * kHalfD;
 #pragma unroll 1
-        for (int i = 0; i < D / 32; ++i) {
+        for (int i = 0; i < kHalfD / 32; ++i) {
           uint32_t o[32];
           tmem_ld32(t_o + 32 * i, o);
           tmem_ld_wait();
           if (row < a.N) {
-            uint32_t h[16];
+            uint32_t hh[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c = 32 * i + 2 * e;
-              h[e] = pack2<OutT>(__fmul_rn(__fmul_rn(u2f(o[2 * e]), __ldg(vs + c)), inv),
-                                 __fmul_rn(__fmul_rn(u2f(o[2 * e + 1]), __ldg(vs + c + 1)), inv));
+              hh[e] = pack2<OutT>(__fdiv_rn(__fmul_rn(u2f(o[2 * e]), __ldg(vs + c)), l),
+                                  __fdiv_rn(__fmul_rn(u2f(o[2 * e + 1]), __ldg(vs + c + 1)), l));
             }
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
               *reinterpret_cast<uint4*>(orow + 32 * i + 8 * v4) =
-                  make_uint4(h[4 * v4], h[4 * v4 + 1], h[4 * v4 + 2], h[4 * v4 + 3]);
+                  make_uint4(hh[4 * v4], hh[4 * v4 + 1], hh[4 * v4 + 2], hh[4 * v4 + 3]);
           }
         }
       }
@@ -382,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -477,10 +617,10 @@ static bool make_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mq, CUten
          (mv == nullptr || make_tmap_u8_3d(mv, w.vt_codes, pb.Npad, pb.d, pb.BH, 128, pb.d));
 }
 
-template <int D, typename OutT>
+template <int D, typename OutT, bool HAS_BIAS>
 static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                             int BH, cudaStream_t s) {
-  auto kern = attn_i8f8_kernel<D, OutT>;
+  auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::alloc);
@@ -506,12 +646,20 @@ cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, floa
   a.causal = pb.causal;
   a.num_pairs = (pb.Npad / 128 + 1) / 2;
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)pb.d));
-  a.Pr = Pr;
-  if (pb.d == 128)
-    return pb.dtype == 0 ? run_attn<128, __half>(mq, mk, mv, a, pb.BH, s)
-                         : run_attn<128, __nv_bfloat16>(mq, mk, mv, a, pb.BH, s);
-  return pb.dtype == 0 ? run_attn<64, __half>(mq, mk, mv, a, pb.BH, s)
-                       : run_attn<64, __nv_bfloat16>(mq, mk, mv, a, pb.BH, s);
+  a.log2Pr = (float)log2((double)Pr);
+  const bool bias = a.bias != nullptr;
+  if (pb.d == 128) {
+    if (pb.dtype == 0)
+      return bias ? run_attn<128, __half, true>(mq, mk, mv, a, pb.BH, s)
+                  : run_attn<128, __half, false>(mq, mk, mv, a, pb.BH, s);
+    return bias ? run_attn<128, __nv_bfloat16, true>(mq, mk, mv, a, pb.BH, s)
+                : run_attn<128, __nv_bfloat16, false>(mq, mk, mv, a, pb.BH, s);
+  }
+  if (pb.dtype == 0)
+    return bias ? run_attn<64, __half, true>(mq, mk, mv, a, pb.BH, s)
+                : run_attn<64, __half, false>(mq, mk, mv, a, pb.BH, s);
+  return bias ? run_attn<64, __nv_bfloat16, true>(mq, mk, mv, a, pb.BH, s)
+              : run_attn<64, __nv_bfloat16, false>(mq, mk, mv, a, pb.BH, s);
 }
 
 cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s) {

@@ -293,7 +293,34 @@ def test_dropping_the_rescale_is_caught():
     ptil = np.vectorize(lambda x: orc.e4m3_decode(orc.e4m3_encode(x)))(np.float32(p * 448.0))
     vdq = np.stack([orc.e4m3_decode_array(qz2["vt_codes"][b, :, :N]).T for b in range(2)])
     o_plain = (ptil @ vdq) * qz2["v_scale"][:, None, :] / (448.0 * p.sum(axis=2, keepdims=True))
-    assert np.max(np.abs(o2[:, rows] - o_plain[:, rows])) < 2e-5
+    # exact 2^x here vs the oracle's polynomial (within 8.6e-5): the row sums
+    # differ by up to ~1e-4 relative and a P~ code may flip where p*448 sits
+    # that close to a rounding midpoint; a dropped rescale gives errors of the
+    # size of O itself
+    err = np.abs(o2[:, rows] - o_plain[:, rows])
+    assert np.max(err) < 5e-3 and np.mean(err) < 3e-4
+
+
+# The oracle's exp2 (tested against libm below) is within 8.6e-5 of 2^x, and
+# the logit max is subtracted after rounding; single-key and equal-logit rows
+# therefore reproduce V within ~1e-4 relative, not to the last bit.
+EXP2_RTOL = 2e-4
+
+
+def test_exp2_against_libm():
+    """orc_exp2: Cody-Waite reduction + degree-3 polynomial; relative error
+    below 8.6e-5 of the library exp2 over the range the softmax uses, exact at
+    integers, +0 at and below -127 and for NaN, monotonic."""
+    xs = np.concatenate([np.linspace(-126, 9, 400001), np.arange(-126, 10, dtype=np.float64)]).astype(np.float32)
+    got = np.array([orc.exp2(float(x)) for x in xs], np.float64)
+    ref = np.exp2(xs.astype(np.float64))
+    assert np.max(np.abs(got / ref - 1)) < 8.6e-5
+    ints = np.arange(-126, 10)
+    assert all(orc.exp2(float(i)) == 2.0 ** i for i in ints)
+    assert orc.exp2(-127.0) == 0.0 and orc.exp2(float("-inf")) == 0.0 and orc.exp2(-500.0) == 0.0
+    assert orc.exp2(float("nan")) == 0.0
+    g = np.array([orc.exp2(float(x)) for x in np.linspace(-20, 9, 100001, dtype=np.float32)])
+    assert np.all(np.diff(g) >= 0)
 
 
 def test_single_key_returns_dequantized_v():
@@ -302,7 +329,7 @@ def test_single_key_returns_dequantized_v():
         qz = orc.quantize_int8_fp8(q, k, v, False, mode)
         o = orc.attention_int8_fp8(qz, False)
         vdq = orc.e4m3_decode_array(qz["vt_codes"][:, :, 0]) * qz["v_scale"]
-        assert np.allclose(o[:, 0], vdq, rtol=2e-7, atol=0)
+        assert np.allclose(o[:, 0], vdq, rtol=EXP2_RTOL, atol=0)
 
 
 def test_zero_q_gives_mean_of_dequantized_v():
@@ -312,11 +339,12 @@ def test_zero_q_gives_mean_of_dequantized_v():
     o = orc.attention_int8_fp8(qz, False)
     vdq = np.stack([orc.e4m3_decode_array(qz["vt_codes"][b, :, :300]).T for b in range(2)])
     mean = (vdq * qz["v_scale"][:, None, :]).mean(axis=1)
-    assert np.allclose(o, mean[:, None, :], rtol=1e-5, atol=1e-6)
+    assert np.allclose(o, mean[:, None, :], rtol=EXP2_RTOL, atol=1e-6)
     # causal: row 0 sees only key 0
     oc = orc.attention_int8_fp8(qz, True)
-    assert np.allclose(oc[:, 0], vdq[:, 0] * qz["v_scale"], rtol=2e-7, atol=0)
-    assert np.allclose(oc[:, 9], (vdq[:, :10] * qz["v_scale"][:, None, :]).mean(axis=1), rtol=1e-5, atol=1e-6)
+    assert np.allclose(oc[:, 0], vdq[:, 0] * qz["v_scale"], rtol=EXP2_RTOL, atol=0)
+    assert np.allclose(oc[:, 9], (vdq[:, :10] * qz["v_scale"][:, None, :]).mean(axis=1), rtol=EXP2_RTOL,
+                       atol=1e-6)
 
 
 def test_pages_fp16_range_pairs():
@@ -342,7 +370,7 @@ def test_f16acc_worst_case_stays_finite_and_wider_range_overflows():
     qz = orc.quantize_int8_fp8(q, k, v, False, orc.MODE_INT8_FP8_F16ACC)
     assert np.all(orc.e4m3_decode_array(qz["vt_codes"][:, :, :N]) == 4.5)
     o = orc.attention_int8_fp8(qz, False)
-    assert np.all(np.isfinite(o)) and np.allclose(o, 2.0, rtol=1e-6)
+    assert np.all(np.isfinite(o)) and np.allclose(o, 2.0, rtol=EXP2_RTOL)
     vt9, sv9 = orc.quant_v_fp8(v, orc.channel_absmax(v), 9.0)
     qz9 = dict(qz, vt_codes=vt9, v_scale=sv9)
     o9 = orc.attention_int8_fp8(qz9, False)
