@@ -52,8 +52,8 @@ struct Smem {
   static constexpr int off_q = 0;
   static constexpr int off_k = off_q + 2 * kQ;
   static constexpr int off_v = off_k + kStages * kK;
-  static constexpr int off_p = off_v + kStages * kV;
-  static constexpr int off_bar = off_p + 2 * kP;
+  static constexpr int off_p = off_v + kStages * kV;  // [query tile 2][buffer 2]
+  static constexpr int off_bar = off_p + 4 * kP;
   // row-max / row-sum exchange between the two key halves:
   // [query tile 2][tile parity 2][half 2][row 128] floats
   static constexpr int off_x = off_bar + 256;
@@ -97,36 +97,54 @@ SAGE_DEV float fmax3(float a, float b, float c) {
   return d;
 }
 
-// exp2 of the method, the same definition the CPU reference computation uses:
-// d clamped to -127 (NaN included), d = n + f with n = floor(d) (the
-// round-down add of 1.5*2^23 gives 1.5*2^23 + n exactly), 2^f by a degree-3
-// polynomial with constant term 1 (Remez fit of the relative error, max
-// 8.6e-5), then n added to the exponent field.  2^(integer) is exact; d <= -127
-// gives +0.
+// exp2 of the method, the same definition the CPU reference computation uses.
+// The argument is carried as g = (d + 127) / 256 saturated to [0, 1]; then
+// k = floor(256 g) (the round-down fma with 1.5*2^23 - 127 gives
+// 1.5*2^23 - 127 + k exactly), f = 256 g - k, 2^f by a degree-3 polynomial
+// with constant term 1 (Remez fit of the relative error, max 8.6e-5), and
+// k - 127 added to the exponent field.  Exact at integer d; d <= -127 gives +0.
 constexpr float kE1 = 0x1.63e658p-1f, kE2 = 0x1.d2378ap-3f, kE3 = 0x1.3baaa6p-4f;
+constexpr float kMg = 12582912.0f - 127.0f;
 
-SAGE_DEV float exp2m(float d) {
-  d = fmaxf(d, -127.0f);
-  const float y = __fadd_rd(d, kMagicF);
-  const float f = __fadd_rn(d, -__fadd_rn(y, -kMagicF));
+SAGE_DEV float sat_fma(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+SAGE_DEV float exp2g(float g) {
+  const float y = __fmaf_rd(g, 256.0f, kMg);
+  const float f = __fmaf_rn(g, 256.0f, -__fadd_rn(y, -kMg));
   float r = __fmaf_rn(kE3, f, kE2);
   r = __fmaf_rn(r, f, kE1);
   r = __fmaf_rn(r, f, 1.0f);
   return __uint_as_float(__float_as_uint(r) + (__float_as_uint(y) << 23));
 }
 
-// The same on a pair, with the packed f32x2 ALU operations.
-SAGE_DEV float2 exp2m2(float2 d) {
-  d.x = fmaxf(d.x, -127.0f);
-  d.y = fmaxf(d.y, -127.0f);
-  const float2 y = __fadd2_rd(d, make_float2(kMagicF, kMagicF));
-  const float2 n = __fadd2_rn(y, make_float2(-kMagicF, -kMagicF));
-  const float2 f = __fadd2_rn(d, make_float2(-n.x, -n.y));
+// exp2 of a plain argument d (used for the rescale factor alpha).
+SAGE_DEV float exp2m(float d) { return exp2g(__saturatef(__fmul_rn(__fadd_rn(d, 127.0f), 0x1p-8f))); }
+
+// The same as exp2g on a pair, with the packed f32x2 ALU operations.
+SAGE_DEV float2 exp2g2(float2 g) {
+  const float2 y = __ffma2_rd(g, make_float2(256.0f, 256.0f), make_float2(kMg, kMg));
+  const float2 k = __fadd2_rn(y, make_float2(-kMg, -kMg));
+  const float2 f = __ffma2_rn(g, make_float2(256.0f, 256.0f), make_float2(-k.x, -k.y));
   float2 r = __ffma2_rn(make_float2(kE3, kE3), f, make_float2(kE2, kE2));
   r = __ffma2_rn(r, f, make_float2(kE1, kE1));
   r = __ffma2_rn(r, f, make_float2(1.0f, 1.0f));
   return make_float2(__uint_as_float(__float_as_uint(r.x) + (__float_as_uint(y.x) << 23)),
                      __uint_as_float(__float_as_uint(r.y) + (__float_as_uint(y.y) << 23)));
+}
+
+// Four floats -> four e4m3 codes in one word (round to nearest even,
+// saturate to +-448); a.x lands in the low byte.
+SAGE_DEV uint32_t e4m3x4(float2 a, float2 b) {
+  uint32_t w;
+  asm("{\n\t.reg .b16 lo, hi;\n\tcvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\tmov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(w)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return w;
 }
 
 SAGE_DEV float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(&s_full[q]);
       };
       auto issue_pv = [&](int q, int j) {
-        const uint32_t pa = p_base + q * L::kP, vb = v_base + (j % kStages) * L::kV;
+        const uint32_t pa = p_base + (2 * q + (j & 1)) * L::kP, vb = v_base + (j % kStages) * L::kV;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f8(tmem + 256 + q * D, kmajor_desc(pa + kk * 32, 128), kmajor_desc(vb + kk * 32, 128), idesc_pv,
@@ -326,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
       const uint32_t t_s = tmem + lane_off + q * 128 + h * 64;
       const uint32_t t_o = tmem + lane_off + 256 + q * D + h * kHalfD;
-      uint8_t* prow = smem + L::off_p + q * L::kP + r * 128;
+      uint8_t* prow0 = smem + L::off_p + 2 * q * L::kP + r * 128;  // buffer 0; buffer 1 is kP further
       const float* ksc = a.k_scale + (size_t)bh * (a.Npad / 64);
       const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
       float* xq = xch + q * 512;  // [parity][half][row]
@@ -334,7 +352,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
       bool ok = true;
+      // K scales of both 64-key granules of the tile, loaded one tile ahead
+      float2 ks_next = *reinterpret_cast<const float2*>(ksc);
       for (int j = 0; j < nt[q]; ++j) {
+        const float2 ks = ks_next;
+        if (j + 1 < nt[q]) ks_next = *reinterpret_cast<const float2*>(ksc + 2 * (j + 1));
+        const int kbase = j * 128 + h * 64;
+        // visible keys of this row among the half's 64 form the prefix c < lim
+        int lim = 64;
+        if (kbase + 63 >= a.N || (a.causal && j == qt)) {
+          lim = min(lim, a.N - kbase);
+          if (a.causal) lim = min(lim, row - kbase + 1);
+        }
         // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
         if (!__all_sync(0xffffffffu, mbar_wait(&s_full[q], j & 1, abort_flag))) {
           ok = false;
@@ -353,28 +382,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // reference computation takes the same ones):
         //   kf = (sq * sk) * log2(e)/sqrt(d) for this half's 64-key granule,
         //   t  = float(S) * kf  (or fma(float(S), kf, bias * log2(e)/sqrt(d))),
-        //   m' = max - log2(Pr),  d = fma(float(S), kf, -m')  (or t - m'),
-        //   p' = exp2m(d) = p * Pr,  P~ = e4m3(p').
-        const float kf = __fmul_rn(__fmul_rn(sq, ksc[2 * j + h]), a.c_log2);
-        const int kbase = j * 128 + h * 64;
-        // visible keys of this row among the half's 64 form the prefix c < lim
-        int lim = 64;
-        if (kbase + 63 >= a.N || (a.causal && j == qt)) {
-          lim = min(lim, a.N - kbase);
-          if (a.causal) lim = min(lim, row - kbase + 1);
-        }
-        // S + 1.5*2^23 read as a float is exactly 1.5*2^23 + S (|S| < 2^22),
-        // and positive floats order like their integers.  Masked keys become
-        // -inf: below every biased value in the max, and d = -inf (or NaN
-        // for a zero scale) clamps to -127, where exp2m gives +0.
+        //   m' = max - log2(Pr),  g = sat(fma(float(S), kf/256, (127 - m')/256))
+        //   (or sat(fma(t, 1/256, (127 - m')/256))),  p' = exp2g(g) = p * Pr,
+        //   P~ = e4m3(p').
+        // Masked keys become -inf: out of the max, and g saturates to 0 (also
+        // from NaN, for a zero scale), where exp2g gives +0.
+        const float kf = __fmul_rn(__fmul_rn(sq, h ? ks.y : ks.x), a.c_log2);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) sr[c] += kMagicI;
+        for (int c = 0; c < 64; ++c) sr[c] = f2u(__int2float_rn((int)sr[c]));
         if (lim < 64) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if (c >= lim) sr[c] = 0xFF800000u;
         }
-        const float2 nmag = make_float2(-kMagicF, -kMagicF);
         float mt;
         if (!HAS_BIAS) {
           float ga = -INFINITY, gb = -INFINITY;
@@ -384,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             gb = fmax3(gb, u2f(sr[c + 2]), u2f(sr[c + 3]));
           }
           // a half with no visible key gives -inf, or NaN for a zero scale
-          mt = __fmul_rn(fmaxf(ga, gb) - kMagicF, kf);
+          mt = __fmul_rn(fmaxf(ga, gb), kf);
         } else {
           const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
@@ -393,10 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c4 = 0; c4 < 16; ++c4) {
             const float4 bv = __ldg(b4 + c4);
             const int c = 4 * c4;
-            const float2 xa = __fadd2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), nmag);
-            const float2 xb = __fadd2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), nmag);
-            const float2 ta = __ffma2_rn(xa, make_float2(kf, kf), __fmul2_rn(make_float2(bv.x, bv.y), cl2));
-            const float2 tb = __ffma2_rn(xb, make_float2(kf, kf), __fmul2_rn(make_float2(bv.z, bv.w), cl2));
+            const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
+                                         __fmul2_rn(make_float2(bv.x, bv.y), cl2));
+            const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf),
+                                         __fmul2_rn(make_float2(bv.z, bv.w), cl2));
             sr[c] = f2u(ta.x);
             sr[c + 1] = f2u(ta.y);
             sr[c + 2] = f2u(tb.x);
@@ -417,33 +437,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mt = fmaxf(mt, xs[(h ^ 1) * 128 + r]);
         const float m_new = fmaxf(m, mt);
-        const float alpha = exp2m(m - m_new);  // +0 on the first tile (m = -inf), 1 if the max stays
+        const float alpha = exp2m(__fadd_rn(m, -m_new));  // +0 on the first tile (m = -inf), 1 if the max stays
         const float mp = m_new - a.log2Pr;
+        const float cs = __fmul_rn(__fadd_rn(127.0f, -mp), 0x1p-8f);
+        const float gm = HAS_BIAS ? 0x1p-8f : __fmul_rn(kf, 0x1p-8f);
 
-        // p' = p * Pr for the 64 keys, P~ = e4m3(p') packed 4 per word, and
-        // the sum of p'
-        uint32_t pw[16];
+        // p' = p * Pr for the 64 keys, P~ = e4m3(p') packed 4 per word and
+        // stored 16 keys at a time into this tile's P buffer (the buffer was
+        // last read by the P~V two tiles back, which completed before the
+        // previous tile's rescale), and the sum of p'
+        uint8_t* prow = prow0 + (j & 1) * L::kP;
         float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-        const float2 nmp = make_float2(-mp, -mp), kf2 = make_float2(kf, kf);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const int c = 4 * c4;
-          float2 da, db;
-          if (!HAS_BIAS) {
-            da = __ffma2_rn(__fadd2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), nmag), kf2, nmp);
-            db = __ffma2_rn(__fadd2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), nmag), kf2, nmp);
-          } else {
-            da = __fadd2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), nmp);
-            db = __fadd2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), nmp);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t pw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 16 * cc + 4 * e;
+            const float2 ga2 = make_float2(sat_fma(u2f(sr[c]), gm, cs), sat_fma(u2f(sr[c + 1]), gm, cs));
+            const float2 gb2 = make_float2(sat_fma(u2f(sr[c + 2]), gm, cs), sat_fma(u2f(sr[c + 3]), gm, cs));
+            const float2 pa = exp2g2(ga2), pb = exp2g2(gb2);
+            sa = __fadd2_rn(sa, pa);
+            sb = __fadd2_rn(sb, pb);
+            pw[e] = e4m3x4(pa, pb);
           }
-          const float2 pa = exp2m2(da), pb = exp2m2(db);
-          sa = __fadd2_rn(sa, pa);
-          sb = __fadd2_rn(sb, pb);
-          pw[c4] = (uint32_t)e4m3x2(pa.x, pa.y) | ((uint32_t)e4m3x2(pb.x, pb.y) << 16);
+          *reinterpret_cast<uint4*>(prow + (((4 * h + cc) ^ (r & 7)) << 4)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
+        fence_proxy_async_smem();
         if (j > 0) {
-          // P~V of the previous tile must be done: its P buffer is reused and
-          // its O rows are rescaled below.
+          // P~V of the previous tile must be done before its O rows are
+          // rescaled (and before the next tile reuses that P buffer).
           if (!__all_sync(0xffffffffu, mbar_wait(&o_done[q], (j - 1) & 1, abort_flag))) {
             ok = false;
             break;
@@ -466,11 +489,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
           }
         }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          *reinterpret_cast<uint4*>(prow + (((4 * h + cc) ^ (r & 7)) << 4)) =
-              make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[q]);

@@ -54,17 +54,29 @@ SAGE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same, but the thread may sleep up to `hint_ns` while the phase is
+// incomplete (it wakes when the phase completes), so waiting costs no issue slots.
+SAGE_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, "
+      "p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait for the phase with the given parity.  `abort` points to a
 // CTA-shared flag; once another role has given up, the wait stops early.
+// Each poll sleeps up to 100 us, so the loop runs a few tens of thousands of
+// times at most before the time limit.
 SAGE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_ns();
-  for (uint32_t it = 1; it < SAGE_SPIN_LIMIT; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort) return false;
-      if (global_ns() - t0 > SAGE_WAIT_NS) return false;
-    }
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 0; it < SAGE_SPIN_LIMIT; ++it) {
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > SAGE_WAIT_NS) return false;
   }
   return false;
 }

@@ -308,13 +308,14 @@ EXP2_RTOL = 2e-4
 
 
 def test_exp2_against_libm():
-    """orc_exp2: Cody-Waite reduction + degree-3 polynomial; relative error
-    below 8.6e-5 of the library exp2 over the range the softmax uses, exact at
-    integers, +0 at and below -127 and for NaN, monotonic."""
+    """orc_exp2: argument (d + 127)/256 saturated to [0, 1], range reduction,
+    degree-3 polynomial; relative error below 8.6e-5 (polynomial) + 5.3e-6
+    (rounding of d + 127) of the library exp2 over the range the softmax uses,
+    exact at integers, +0 at and below -127 and for NaN, monotonic."""
     xs = np.concatenate([np.linspace(-126, 9, 400001), np.arange(-126, 10, dtype=np.float64)]).astype(np.float32)
     got = np.array([orc.exp2(float(x)) for x in xs], np.float64)
     ref = np.exp2(xs.astype(np.float64))
-    assert np.max(np.abs(got / ref - 1)) < 8.6e-5
+    assert np.max(np.abs(got / ref - 1)) < 8.6e-5 + 5.3e-6
     ints = np.arange(-126, 10)
     assert all(orc.exp2(float(i)) == 2.0 ** i for i in ints)
     assert orc.exp2(-127.0) == 0.0 and orc.exp2(float("-inf")) == 0.0 and orc.exp2(-500.0) == 0.0
