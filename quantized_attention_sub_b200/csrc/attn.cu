@@ -38,22 +38,28 @@ namespace sage {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kSoftmaxWarps = 16;
-constexpr int kProducerWarp = 16, kMmaWarp = 17;
-constexpr int kThreads = 32 * 18;
+// Query tiles per CTA: two with the FP32 accumulator (TMEM S_0, S_1, O_0, O_1),
+// one with the FP16 accumulator (TMEM S, O, H_0, H_1).
+template <bool F16ACC>
+struct Roles {
+  static constexpr int kNQ = F16ACC ? 1 : 2;
+  static constexpr int kSoftmaxWarps = 8 * kNQ;  // two key halves x 4 warps per query tile
+  static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+};
 constexpr uint32_t kTmemCols = 512;
 
-template <int D>
+template <int D, int NQ>
 struct Smem {
   static constexpr int kQ = 128 * D;  // one Q tile (int8)
   static constexpr int kK = 128 * D;  // one K tile (int8)
   static constexpr int kV = D * 128;  // one V^T tile (e4m3)
   static constexpr int kP = 128 * 128;
   static constexpr int off_q = 0;
-  static constexpr int off_k = off_q + 2 * kQ;
+  static constexpr int off_k = off_q + NQ * kQ;
   static constexpr int off_v = off_k + kStages * kK;
-  static constexpr int off_p = off_v + kStages * kV;  // [query tile 2][buffer 2]
-  static constexpr int off_bar = off_p + 4 * kP;
+  static constexpr int off_p = off_v + kStages * kV;  // [query tile NQ][buffer 2]
+  static constexpr int off_bar = off_p + 2 * NQ * kP;
   // row-max / row-sum exchange between the two key halves:
   // [query tile 2][tile parity 2][half 2][row 128] floats
   static constexpr int off_x = off_bar + 256;
@@ -68,7 +74,7 @@ struct AttnArgs {
   const float* bias;  // null unless smooth_q
   void* out;
   int* err;
-  int N, Npad, causal, num_pairs;
+  int N, Npad, causal, num_qblocks;
   float c_log2, log2Pr;
 };
 
@@ -147,6 +153,21 @@ SAGE_DEV uint32_t e4m3x4(float2 a, float2 b) {
   return w;
 }
 
+// 32 lanes x 32 columns whose 32-bit cells each hold one f16 accumulator in
+// the low half: thread t gets 16 registers, register i = columns (2i, 2i+1).
+SAGE_DEV void tmem_ld16_pack16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.pack::16b.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+SAGE_DEV float2 h2f2(uint32_t u) {
+  __half2 h = *reinterpret_cast<__half2*>(&u);
+  return __half22float2(h);
+}
+
 SAGE_DEV float u2f(uint32_t u) { return __uint_as_float(u); }
 SAGE_DEV uint32_t f2u(float f) { return __float_as_uint(f); }
 
@@ -165,11 +186,17 @@ SAGE_DEV uint32_t pack2<__nv_bfloat16>(float a, float b) {
 
 }  // namespace
 
-template <int D, typename OutT, bool HAS_BIAS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, typename OutT, bool HAS_BIAS, bool F16ACC>
+__global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
-  using L = Smem<D>;
+  using R = Roles<F16ACC>;
+  constexpr int kNQ = R::kNQ;
+  constexpr int kSoftmaxWarps = R::kSoftmaxWarps, kProducerWarp = R::kProducerWarp, kMmaWarp = R::kMmaWarp;
+  using L = Smem<D, kNQ>;
+  // TMEM columns: S_q, O_q, and (FP16 accumulator) the two 64-key chunk partials H_c
+  constexpr uint32_t kColO = F16ACC ? 128u : 256u;
+  constexpr uint32_t kColH = 128u + D;
   constexpr int kHalfD = D / 2;  // O columns each key half rescales and stores
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -190,16 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* xch = (float*)(smem + L::off_x);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = a.causal ? (a.num_pairs - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int qb = a.causal ? (a.num_qblocks - 1 - (int)blockIdx.x) : (int)blockIdx.x;
   const int bh = blockIdx.y;
   const int n_ktiles = a.Npad / 128;
-  int nt[2];
+  int nt[kNQ];
+  int T = 0;
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int qt = 2 * pair + q;
+  for (int q = 0; q < kNQ; ++q) {
+    const int qt = kNQ * qb + q;
     nt[q] = qt >= n_ktiles ? 0 : (a.causal ? qt + 1 : n_ktiles);
+    T = max(T, nt[q]);
   }
-  const int T = max(nt[0], nt[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -209,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int q = 0; q < 2; ++q) {
+    for (int q = 0; q < kNQ; ++q) {
       mbar_init(&s_full[q], 1);
       mbar_init(&s_free[q], 8);   // 8 softmax warps per query tile
       mbar_init(&p_full[q], 8);
@@ -236,10 +264,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      const uint32_t qbytes = (nt[0] > 0 ? L::kQ : 0) + (nt[1] > 0 ? L::kQ : 0);
+      uint32_t qbytes = 0;
+      for (int q = 0; q < kNQ; ++q) qbytes += nt[q] > 0 ? L::kQ : 0;
       mbar_arrive_expect_tx(q_full, qbytes);
-      for (int q = 0; q < 2; ++q)
-        if (nt[q] > 0) tma_load_3d(smem + L::off_q + q * L::kQ, &tm_q, q_full, 0, (2 * pair + q) * 128, bh);
+      for (int q = 0; q < kNQ; ++q)
+        if (nt[q] > 0) tma_load_3d(smem + L::off_q + q * L::kQ, &tm_q, q_full, 0, (kNQ * qb + q) * 128, bh);
       int issued_k = 0, issued_v = 0;
       for (int j = 0; j < T; ++j) {
         const int s = j % kStages, n = j / kStages;
@@ -270,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_make(2u, 1u, 1u, 128, 128);  // s32 <- s8 x s8
-      constexpr uint32_t idesc_pv = idesc_make(1u, 0u, 0u, 128, D);   // f32 <- e4m3 x e4m3
+      // P~V: f32 <- e4m3 x e4m3, or f16 <- e4m3 x e4m3 per 64-key chunk
+      constexpr uint32_t idesc_pv = idesc_make(F16ACC ? 0u : 1u, 0u, 0u, 128, D);
       const uint32_t q_base = smem_u32(smem + L::off_q), k_base = smem_u32(smem + L::off_k);
       const uint32_t v_base = smem_u32(smem + L::off_v), p_base = smem_u32(smem + L::off_p);
       bool ok = mbar_wait(q_full, 0, abort_flag);
@@ -283,16 +313,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int q, int j) {
         const uint32_t pa = p_base + (2 * q + (j & 1)) * L::kP, vb = v_base + (j % kStages) * L::kV;
+        if (F16ACC) {
+          // keys [64c, 64c + 64) into H_c: two k = 32 steps accumulated in f16
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8(tmem + 256 + q * D, kmajor_desc(pa + kk * 32, 128), kmajor_desc(vb + kk * 32, 128), idesc_pv,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8(tmem + kColH + (kk >> 1) * D, kmajor_desc(pa + kk * 32, 128), kmajor_desc(vb + kk * 32, 128),
+                   idesc_pv, kk & 1);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8(tmem + kColO + q * D, kmajor_desc(pa + kk * 32, 128), kmajor_desc(vb + kk * 32, 128), idesc_pv,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+        }
         tc_commit(&o_done[q]);
       };
       if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        for (int q = 0; q < 2; ++q)
+        for (int q = 0; q < kNQ; ++q)
           if (nt[q] > 0) issue_s(q, 0);
         tc_commit(&k_empty[0]);
       }
@@ -304,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         // next S tiles first (they need only the S buffers back), then P~V
-        for (int q = 0; q < 2 && ok; ++q) {
+        for (int q = 0; q < kNQ && ok; ++q) {
           if (j + 1 < nt[q]) {
             if (!(ok = mbar_wait(&s_free[q], j & 1, abort_flag))) break;
             tc_fence_after();
@@ -315,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (next_k) tc_commit(&k_empty[(j + 1) % kStages]);
         if (!(ok = mbar_wait(&v_full[j % kStages], (j / kStages) & 1, abort_flag))) break;
         tc_fence_after();
-        for (int q = 0; q < 2 && ok; ++q) {
+        for (int q = 0; q < kNQ && ok; ++q) {
           if (j < nt[q]) {
             if (!(ok = mbar_wait(&p_full[q], j & 1, abort_flag))) break;
             tc_fence_after();
@@ -338,12 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = threadIdx.x & 127;
     const int w4 = warp & 3;
     if (nt[q] > 0) {
-      const int qt = 2 * pair + q;
+      const int qt = kNQ * qb + q;
       const int row = qt * 128 + r;
       const float sq = a.q_scale[(size_t)bh * (a.Npad / 32) + (row >> 5)];
       const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
       const uint32_t t_s = tmem + lane_off + q * 128 + h * 64;
-      const uint32_t t_o = tmem + lane_off + 256 + q * D + h * kHalfD;
+      const uint32_t t_o = tmem + lane_off + kColO + q * D + h * kHalfD;
+      const uint32_t t_h = tmem + lane_off + kColH + h * kHalfD;  // H_0 here, H_1 is D columns further
       uint8_t* prow0 = smem + L::off_p + 2 * q * L::kP + r * 128;  // buffer 0; buffer 1 is kP further
       const float* ksc = a.k_scale + (size_t)bh * (a.Npad / 64);
       const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
@@ -351,7 +390,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // m: running row max of the logits (log2 units); l: this half's running
       // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
+      float alpha_prev = 0.f;  // FP16 accumulator: rescale factor of the tile whose partials are pending
       bool ok = true;
+      // FP16 accumulator, after P~V(jt) completed: acc = (alpha_jt * acc + h_0) + h_1
+      // over this half's O columns (the first tile starts from acc = 0).
+      auto fold_partials = [&](int jt, float alpha_t) {
+#pragma unroll 1
+        for (int i = 0; i < kHalfD / 32; ++i) {
+          uint32_t o[32], h0[16], h1[16];
+          tmem_ld16_pack16(t_h + 32 * i, h0);
+          tmem_ld16_pack16(t_h + D + 32 * i, h1);
+          if (jt > 0) tmem_ld32(t_o + 32 * i, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float2 acc = jt > 0 ? __fmul2_rn(make_float2(u2f(o[2 * e]), u2f(o[2 * e + 1])), make_float2(alpha_t, alpha_t))
+                                : make_float2(0.f, 0.f);
+            acc = __fadd2_rn(__fadd2_rn(acc, h2f2(h0[e])), h2f2(h1[e]));
+            o[2 * e] = f2u(acc.x);
+            o[2 * e + 1] = f2u(acc.y);
+          }
+          tmem_st32(t_o + 32 * i, o);
+        }
+        tmem_st_wait();
+      };
       // K scales of both 64-key granules of the tile, loaded one tile ahead
       float2 ks_next = *reinterpret_cast<const float2*>(ksc);
       for (int j = 0; j < nt[q]; ++j) {
@@ -472,7 +534,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          if (F16ACC) {
+            // fold the previous tile's FP16 partials into the FP32 accumulator
+            // before this tile's P~V overwrites them
+            fold_partials(j - 1, alpha_prev);
+          } else if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
             for (int i = 0; i < kHalfD / 32; ++i) {
               uint32_t o[32];
@@ -494,8 +560,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[q]);
         l = __fadd_rn(__fmul_rn(alpha, l), (sa.x + sa.y) + (sb.x + sb.y));
         m = m_new;
+        alpha_prev = alpha;
       }
       if (ok && !__all_sync(0xffffffffu, mbar_wait(&o_done[q], (nt[q] - 1) & 1, abort_flag))) ok = false;
+      if (ok && F16ACC) {
+        tc_fence_after();
+        fold_partials(nt[q] - 1, alpha_prev);
+      }
       if (ok) {
         // the row sum is the sum of both halves' sums
         const int jx = nt[q];
@@ -635,17 +706,18 @@ static bool make_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mq, CUten
          (mv == nullptr || make_tmap_u8_3d(mv, w.vt_codes, pb.Npad, pb.d, pb.BH, 128, pb.d));
 }
 
-template <int D, typename OutT, bool HAS_BIAS>
+template <int D, typename OutT, bool HAS_BIAS, bool F16ACC>
 static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                             int BH, cudaStream_t s) {
-  auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS>;
+  auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS, F16ACC>;
+  using L = Smem<D, Roles<F16ACC>::kNQ>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::alloc);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<dim3(a.num_pairs, BH), kThreads, Smem<D>::alloc, s>>>(mq, mk, mv, a);
+  kern<<<dim3(a.num_qblocks, BH), Roles<F16ACC>::kThreads, L::alloc, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -662,22 +734,20 @@ cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, floa
   a.N = pb.N;
   a.Npad = pb.Npad;
   a.causal = pb.causal;
-  a.num_pairs = (pb.Npad / 128 + 1) / 2;
+  const bool f16 = pb.mode == 1;
+  const int nq = f16 ? 1 : 2;
+  a.num_qblocks = (pb.Npad / 128 + nq - 1) / nq;
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)pb.d));
   a.log2Pr = (float)log2((double)Pr);
   const bool bias = a.bias != nullptr;
-  if (pb.d == 128) {
-    if (pb.dtype == 0)
-      return bias ? run_attn<128, __half, true>(mq, mk, mv, a, pb.BH, s)
-                  : run_attn<128, __half, false>(mq, mk, mv, a, pb.BH, s);
-    return bias ? run_attn<128, __nv_bfloat16, true>(mq, mk, mv, a, pb.BH, s)
-                : run_attn<128, __nv_bfloat16, false>(mq, mk, mv, a, pb.BH, s);
-  }
-  if (pb.dtype == 0)
-    return bias ? run_attn<64, __half, true>(mq, mk, mv, a, pb.BH, s)
-                : run_attn<64, __half, false>(mq, mk, mv, a, pb.BH, s);
-  return bias ? run_attn<64, __nv_bfloat16, true>(mq, mk, mv, a, pb.BH, s)
-              : run_attn<64, __nv_bfloat16, false>(mq, mk, mv, a, pb.BH, s);
+#define SAGE_RUN(DD, TT, BB, FF) run_attn<DD, TT, BB, FF>(mq, mk, mv, a, pb.BH, s)
+#define SAGE_RUN_F(DD, TT, BB) (f16 ? SAGE_RUN(DD, TT, BB, true) : SAGE_RUN(DD, TT, BB, false))
+#define SAGE_RUN_B(DD, TT) (bias ? SAGE_RUN_F(DD, TT, true) : SAGE_RUN_F(DD, TT, false))
+  if (pb.d == 128) return pb.dtype == 0 ? SAGE_RUN_B(128, __half) : SAGE_RUN_B(128, __nv_bfloat16);
+  return pb.dtype == 0 ? SAGE_RUN_B(64, __half) : SAGE_RUN_B(64, __nv_bfloat16);
+#undef SAGE_RUN_B
+#undef SAGE_RUN_F
+#undef SAGE_RUN
 }
 
 cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s) {

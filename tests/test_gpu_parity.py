@@ -127,28 +127,34 @@ def to_dtype_np(x, dtype):
 
 
 ATTN_SMALL = [
-    # (N, d, dtype, law, smooth_q, causal)
-    (128, 64, "fp16", "k_bias", False, False),
-    (1, 128, "bf16", "k_bias", False, False),
-    (33, 64, "fp16", "k_bias", False, True),
-    (129, 128, "bf16", "k_bias_outlier", False, True),
-    (333, 128, "fp16", "qk_bias", True, False),
-    (640, 64, "bf16", "qk_bias", True, True),
-    (1000, 128, "bf16", "k_bias_outlier", False, True),
-    (1000, 128, "fp16", "k_bias", False, False),
+    # (N, d, dtype, law, smooth_q, causal, mode)
+    (128, 64, "fp16", "k_bias", False, False, 0),
+    (1, 128, "bf16", "k_bias", False, False, 0),
+    (33, 64, "fp16", "k_bias", False, True, 0),
+    (129, 128, "bf16", "k_bias_outlier", False, True, 0),
+    (333, 128, "fp16", "qk_bias", True, False, 0),
+    (640, 64, "bf16", "qk_bias", True, True, 0),
+    (1000, 128, "bf16", "k_bias_outlier", False, True, 0),
+    (1000, 128, "fp16", "k_bias", False, False, 0),
+    # FP16 PV accumulator (SageAttention2++)
+    (1, 128, "fp16", "qk_bias", True, False, 1),
+    (128, 64, "fp16", "k_bias", False, False, 1),
+    (200, 128, "fp16", "qk_bias", True, True, 1),
+    (700, 128, "fp16", "qk_bias", True, False, 1),
+    (1000, 64, "bf16", "k_bias_outlier", False, True, 1),
 ]
 
 
-@pytest.mark.parametrize("N,d,dtype,law,smooth_q,causal", ATTN_SMALL)
-def test_attention_matches_oracle(N, d, dtype, law, smooth_q, causal):
-    w = small_workload(N, d, dtype, law, smooth_q, 0, causal=causal)
+@pytest.mark.parametrize("N,d,dtype,law,smooth_q,causal,mode", ATTN_SMALL)
+def test_attention_matches_oracle(N, d, dtype, law, smooth_q, causal, mode):
+    w = small_workload(N, d, dtype, law, smooth_q, mode, causal=causal)
     q, k, v = [t.cuda() for t in inputs.generate(w)]
     B, H = 1, 2
-    ws = api.alloc_workspace(B, H, N, d, 0)
+    ws = api.alloc_workspace(B, H, N, d, mode)
     out = torch.empty_like(q)
-    api.sage_attn_fwd(q, k, v, out, B, H, N, d, causal, 0, api.DTYPE_CODE[q.dtype], smooth_q, ws, ws.numel())
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, causal, mode, api.DTYPE_CODE[q.dtype], smooth_q, ws, ws.numel())
     api.sage_check(ws, ws.numel())
-    oz = oracle_quant((q, k, v), 0, smooth_q)
+    oz = oracle_quant((q, k, v), mode, smooth_q)
     ref = to_dtype_np(orc.attention_int8_fp8(oz, causal), dtype)
     got = out.float().cpu().reshape(B * H, N, d).numpy()
     compare_out(got, ref, dtype, (N, d, dtype, causal))
@@ -174,6 +180,26 @@ def test_full_size_llm_prefill_sampled_rows():
     ref = to_dtype_np(orc.attention_int8_fp8(oz, True, rows=rows), "bf16")
     got = out.float().cpu().reshape(B * H, N, d).numpy()[:, rows]
     compare_out(got, ref, "bf16", "llm_prefill")
+
+
+def test_full_size_video_dit_sampled_rows():
+    """B1 H12 N32760 d128 fp16, non-causal, FP16 PV accumulator, Q smoothing:
+    quantization bit-exact everywhere, the output on sampled rows per head."""
+    w = inputs.WORKLOADS["video_dit"]
+    B, H, N, d = w.shape()
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    ws = api.alloc_workspace(B, H, N, d, w.mode)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, False, w.mode, 0, True, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    g = {n: t.cpu().numpy() for n, t in api.ws_views(ws, B, H, N, d, w.mode).items()}
+    oz = oracle_quant((q, k, v), w.mode, True)
+    assert_quant_bitexact(g, oz, True)
+    rng = np.random.default_rng(32760)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 121, N - 120, N - 1], rng.integers(0, N, 10)])).astype(np.int32)
+    ref = to_dtype_np(orc.attention_int8_fp8(oz, False, rows=rows), "fp16")
+    got = out.float().cpu().reshape(B * H, N, d).numpy()[:, rows]
+    compare_out(got, ref, "fp16", "video_dit")
 
 
 def test_repeated_calls_identical_and_no_error():
