@@ -210,20 +210,20 @@ def main():
     stream = torch.cuda.current_stream()
 
     def step():
+        ev_q.record(stream)
         api.sage_quantize_qkv(q, k, v, dcode, B, H, N, d, w.smooth_q, w.mode, wsbuf, nbytes, stream)
         ev_a.record(stream)
         api.sage_attn_quantized(wsbuf, nbytes, out, dcode, B, H, N, d, w.causal, w.smooth_q, w.mode, stream)
         ev_b.record(stream)
 
-    ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_q, ev_a, ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     for _ in range(args.warmup):
         step()
     api.sage_check(wsbuf, nbytes, stream)
 
     # timed region: K steps; per-step attention-kernel events on the launch stream
     attn_ms = []
-    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
+    ev_pairs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -232,7 +232,7 @@ def main():
     torch.cuda.synchronize()
     t_start.record(stream)
     for i in range(args.steps):
-        ev_a, ev_b = ev_pairs[i]
+        ev_q, ev_a, ev_b = ev_pairs[i]
         step()
     t_stop.record(stream)
     torch.cuda.synchronize()
@@ -240,9 +240,11 @@ def main():
     clk = clocks.stop()
     api.sage_check(wsbuf, nbytes, stream)
     ms = t_start.elapsed_time(t_stop) / args.steps
-    attn_ms = [a_.elapsed_time(b_) for a_, b_ in ev_pairs]
+    attn_ms = [a_.elapsed_time(b_) for _, a_, b_ in ev_pairs]
+    quant_ms = [q_.elapsed_time(a_) for q_, a_, _ in ev_pairs]
     ms = allreduce_max(ms, ws)
     attn_avg = allreduce_max(float(np.mean(attn_ms)), ws)
+    quant_avg = allreduce_max(float(np.mean(quant_ms)), ws)
 
     ops_visible = inputs.executed_ops(w) * ws
     ops_square = inputs.attention_ops(w) * ws
@@ -257,6 +259,14 @@ def main():
                 "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense FP8/INT8 : BF16 ratio)" % (
                     peak_src, FP8_OVER_BF16),
                 "traffic": None, "attn_ms": attn_avg}
+    # the quantization pass (HBM-bound): 16-bit Q, K, V read once, int8/e4m3
+    # codes written, statistics and scales (small) not counted
+    Np = (N + 127) // 128 * 128
+    q_bytes = 3 * B * H * N * d * 2 + 3 * B * H * Np * d
+    hbm = peaks["hbm_gbs"]
+    quant_line = {"bound": "hbm", "kernel": "quant_pass_kernel (stats) + quant_fold_kernel + quant_pass_kernel (codes)", "ms": quant_avg,
+                  "algorithmic_bytes": q_bytes, "achieved": q_bytes / (quant_avg * 1e-3) / 1e9,
+                  "peak": hbm, "unit": "GB/s", "frac": q_bytes / (quant_avg * 1e-3) / 1e9 / hbm}
 
     # end to end through the C ABI with host buffers (pinned), copies inside the region
     hq, hk, hv = [t.cpu().pin_memory() for t in (q, k, v)]
@@ -293,9 +303,11 @@ def main():
             "config": config_of(w, args, ws),
             "value_square_count": ops_square / (ms * 1e-3) / 1e12,
             "roofline": roofline,
+            "quant_roofline": quant_line,
             "e2e": {"value": ops_visible / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes},
-            "gpu_launches": 6 * args.steps,
+            # per step: the stats, fold and codes quantization kernels and attn_i8f8_kernel
+            "gpu_launches": 4 * args.steps,
             "clocks": clk}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle as orc

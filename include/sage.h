@@ -117,8 +117,9 @@ SAGE_API sage_status sage_quantize_qkv(const void* q, const void* k, const void*
  *        the layout places before `scratch`), 1024-byte aligned; it receives
  *        the same codes, scales, means and bias as the workspace of
  *        sage_quantize_qkv, at the same offsets.
- *   Limit: 3*B*H*(Npad/64)*d + B*H*d floats <= 4 Mi (16 MiB); larger problems
- *   return SAGE_ERR_UNSUPPORTED with the sizes in sage_last_error().
+ *   Limit: 3*B*H*(Npad/64)*d + B*H*d words <= 4 Mi (16 MiB);
+ *   larger problems return SAGE_ERR_UNSUPPORTED with the sizes in
+ *   sage_last_error().
  *   The first call on a device looks up the array's device address once,
  *   with that device current; make that first call before any stream
  *   capture.  All calls share the array: calls that overlap on the GPU (on

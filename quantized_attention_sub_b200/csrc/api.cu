@@ -65,8 +65,8 @@ sage_ws_layout layout_of(int B, int H, int N, int d, int mode) {
   L.k_mean = take(BH * d * sizeof(float));
   L.q_mean = take(BH * d * sizeof(float));
   L.q_bias = take(BH * Np * sizeof(float));
-  // statistics partials [3][BH][Np/64][d] and the V multipliers [BH][d]
-  L.scratch = take((3 * BH * (Np / 64) * d + BH * d) * sizeof(float));
+  // statistics partials and V multipliers of the quantize pass
+  L.scratch = take(sage::quant_scratch_floats((int)BH, (int)Np, d) * sizeof(float));
   L.total = off;
   return L;
 }
@@ -193,7 +193,7 @@ sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v
   if (out_bytes < L.scratch)
     return set_err(SAGE_ERR_INVALID_ARG, "output buffer smaller than the layout's quantized region (layout.scratch)%s");
   const size_t Np = ((size_t)N + 127) / 128 * 128, BH = (size_t)B * H;
-  const size_t need = 3 * BH * (Np / 64) * d + BH * d;
+  const size_t need = sage::quant_scratch_floats((int)BH, (int)Np, d);
   if (need > sage::static_scratch_floats()) {
     char buf[200];
     snprintf(buf, sizeof(buf), "problem needs %zu floats of static scratch; the maximum is %zu (16 MiB)", need,

@@ -1,4 +1,4 @@
-// quant.cu -- smoothing and quantization kernels of the INT8/FP8 modes
+// quant.cu -- smoothing and quantization of the INT8/FP8 modes
 // (SageAttention2 abstract: smooth, INT-quantize Q/K, FP8-quantize V;
 // SageAttention2++ summary Sec. 2.1: per-block Q/K scales, per-channel V
 // scales; Sec. 3.1: the narrowed V range Vr).
@@ -15,17 +15,42 @@
 //   bias_n   = fma chain over c of mean_q[c] * k~[n,c]  (smooth_q)
 //   V        : scale_c = a_c / Vr, code = e4m3_rn_satfinite(v * (Vr / a_c))
 //
-// Pass 1 (stats_partials) reads K, V (and Q) once per 64-token chunk and
-// writes per-chunk partial sums / maxima; pass 2 (stats_finalize) folds them
-// per channel; pass 3 (quant_rows / quant_v) reads the inputs again and
-// writes codes.  The three passes are HBM-bound.
+// Three kernels on the stream, none of which waits on another CTA:
+//   stats : per 64-token chunk of each (b, h) slice, the sequential sums of K
+//           (and Q) per channel and the maxima of |V| per channel;
+//   fold  : per slice and tensor, the sequential sum (maximum) over the
+//           chunk partials in chunk order -> means, V scales and multipliers;
+//   codes : per 64-token chunk, K/Q codes and scales, the bias, V codes.
+// The stats and codes kernels are persistent: one loader warp streams each
+// CTA's chunks with TMA into a double buffer while eight compute warps work
+// on the other half.
+//
+// The K and Q granule maxima come from exact packed 16-bit max / min per
+// channel: RN(x - mean) is monotone in x, so the largest |x~| of a channel is
+// the larger of |RN(max - mean)| and |RN(min - mean)|.  Codes use packed fp32
+// adds (each lane rounds like the scalar operation) and take the rounded
+// integer from the low mantissa bits of y + 1.5 * 2^23.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <mutex>
 
 #include "sage_internal.h"
 #include "sage_ptx.cuh"
 
 namespace sage {
+
+namespace {
+
+constexpr int kComputeWarps = 8;
+constexpr int kCompute = 32 * kComputeWarps;  // threads of the compute warps
+constexpr int kThreadsQ = kCompute + 32;      // + one loader warp
+constexpr int kTok = 64;        // tokens per work item (one K granule, two Q granules)
+constexpr int kBoxBytes = 128;  // TMA box row: 64 16-bit channels, SWIZZLE_128B
+constexpr int kBarCompute = 1;  // named barrier of the compute warps
+
+// error code of a CTA whose own tile loads did not land in time
+constexpr int kErrTileWait = 0x202;
 
 template <typename T>
 SAGE_DEV float to_f(T x);
@@ -34,210 +59,633 @@ SAGE_DEV float to_f<__half>(__half x) { return __half2float(x); }
 template <>
 SAGE_DEV float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Four consecutive 16-bit values -> float4.
+// Two 16-bit values packed in a word -> floats (low half first).
 template <typename T>
-SAGE_DEV void load4(const T* p, float* f) {
-  uint2 u = *reinterpret_cast<const uint2*>(p);
-  const T* h = reinterpret_cast<const T*>(&u);
-  f[0] = to_f(h[0]);
-  f[1] = to_f(h[1]);
-  f[2] = to_f(h[2]);
-  f[3] = to_f(h[3]);
+SAGE_DEV void unpack2(uint32_t u, float& lo, float& hi) {
+  T h[2];
+  *reinterpret_cast<uint32_t*>(h) = u;
+  lo = to_f(h[0]);
+  hi = to_f(h[1]);
 }
 
-// ---------------------------------------------------------------- pass 1
-// grid (Npad/64, BH), block D threads; thread c owns channel c of one chunk.
-template <typename T, int D>
-__global__ void __launch_bounds__(D) stats_partials_kernel(const T* __restrict__ k, const T* __restrict__ q,
-                                                           const T* __restrict__ v, int N, int nchunks,
-                                                           float* __restrict__ part) {
-  const int chunk = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-  const int t0 = chunk * 64;
-  const int t1 = min(t0 + 64, N);
-  const size_t base = (size_t)bh * N * D + c;
-  float sk = 0.f, sq = 0.f, av = 0.f;
-  for (int t = t0; t < t1; ++t) {
-    const size_t o = base + (size_t)t * D;
-    sk = __fadd_rn(sk, to_f(k[o]));
-    if (q) sq = __fadd_rn(sq, to_f(q[o]));
-    av = fmaxf(av, fabsf(to_f(v[o])));
+struct QuantArgs {
+  int8_t* q_codes;
+  int8_t* k_codes;
+  uint8_t* vt_codes;
+  float* q_scale;
+  float* k_scale;
+  float* v_scale;
+  float* k_mean;
+  float* q_mean;
+  float* q_bias;
+  float* part;   // [3][BH][Npad/64][d]: K sums, Q sums, |V| maxima per 64-token chunk
+  float* v_mul;  // [BH][d]
+  int* err;
+  int BH, N, Npad, smooth_q, n_items;
+  float Vr;
+};
+
+// Shared-memory image of one 64-token tile of a [.., D] 16-bit tensor as TMA
+// writes it with SWIZZLE_128B: D/64 boxes of 64 rows x 128 bytes, the 16-byte
+// chunk c of row r stored at chunk c ^ (r & 7).  Byte offset of byte `b` of row `r`:
+SAGE_DEV uint32_t swz(int r, int b) {
+  return (uint32_t)((b >> 7) * (kTok * kBoxBytes) + r * kBoxBytes + ((((b >> 4) & 7) ^ (r & 7)) << 4) + (b & 15));
+}
+
+// Packed max / min of two 16-bit values (exact comparisons) and the
+// identities of those reductions.
+template <typename T>
+struct P16;
+template <>
+struct P16<__nv_bfloat16> {
+  static constexpr uint32_t kNegInf = 0xFF80FF80u, kPosInf = 0x7F807F80u;
+  static SAGE_DEV uint32_t max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
   }
-  // part layout: [3][BH][nchunks][D] = sums of K, sums of Q, maxima of |V|
-  const size_t plane = (size_t)gridDim.y * nchunks * D;
-  const size_t o = ((size_t)bh * nchunks + chunk) * D + c;
-  part[o] = sk;
-  part[plane + o] = sq;
-  part[2 * plane + o] = av;
-}
-
-// ---------------------------------------------------------------- pass 2
-// grid BH, block D: channel means in chunk order, V absmax, V scale/multiplier.
-template <int D>
-__global__ void __launch_bounds__(D) stats_finalize_kernel(const float* __restrict__ part, int N, int nchunks,
-                                                           int with_q, float Vr, float* __restrict__ k_mean,
-                                                           float* __restrict__ q_mean, float* __restrict__ v_scale,
-                                                           float* __restrict__ v_mul) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  const int nvalid = (N + 63) / 64;
-  const size_t plane = (size_t)gridDim.x * nchunks * D;
-  float tk = 0.f, tq = 0.f, a = 0.f;
-  for (int g = 0; g < nvalid; ++g) {
-    const size_t o = ((size_t)bh * nchunks + g) * D + c;
-    tk = __fadd_rn(tk, part[o]);
-    if (with_q) tq = __fadd_rn(tq, part[plane + o]);
-    a = fmaxf(a, part[2 * plane + o]);
+  static SAGE_DEV uint32_t min(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
   }
-  k_mean[bh * D + c] = __fdiv_rn(tk, (float)N);
-  if (with_q) q_mean[bh * D + c] = __fdiv_rn(tq, (float)N);
-  v_scale[bh * D + c] = a > 0.f ? __fdiv_rn(a, Vr) : 0.f;
-  v_mul[bh * D + c] = a > 0.f ? __fdiv_rn(Vr, a) : 0.f;
+};
+template <>
+struct P16<__half> {
+  static constexpr uint32_t kNegInf = 0xFC00FC00u, kPosInf = 0x7C007C00u;
+  static SAGE_DEV uint32_t max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  }
+  static SAGE_DEV uint32_t min(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  }
+};
+
+// Low bytes of four floats -> one word (byte i from z[i]).
+SAGE_DEV uint32_t low_bytes4(float z0, float z1, float z2, float z3) {
+  const uint32_t lo = __byte_perm(__float_as_uint(z0), __float_as_uint(z1), 0x0040);
+  const uint32_t hi = __byte_perm(__float_as_uint(z2), __float_as_uint(z3), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
 }
 
-// ---------------------------------------------------------------- pass 3a
-// INT8 quantization of 64 tokens of Q or K: grid (Npad/64, BH), 256 threads.
-// G = granule (32 for Q, 64 for K).  mean may be null (no smoothing).  When
-// bias_mq is set (K with smooth_q), also writes bias[n] for the 64 tokens.
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) quant_rows_int8_kernel(const T* __restrict__ x, const float* __restrict__ mean,
-                                                              int N, int Npad, int8_t* __restrict__ codes,
-                                                              float* __restrict__ scale,
-                                                              const float* __restrict__ bias_mq,
-                                                              float* __restrict__ bias) {
-  constexpr int kRows = 64, kVec = D / 4, kNG = kRows / G;
-  __shared__ float xs[kRows][D + 1];
-  __shared__ float wmax[8][kNG];
-  __shared__ float ginv[kNG];
-  __shared__ float smq[D];
-  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int t0 = blk * kRows;
+// 1.5 * 2^23: for |y| < 2^22, y + kRound rounds y to an integer (ties to
+// even) and leaves it, in two's complement, in the low mantissa bits.
+constexpr float kRound = 12582912.0f;
 
-  float amax0 = 0.f, amax1 = 0.f;  // the block's one or two granules
-  for (int e = tid; e < kRows * kVec; e += 256) {
-    const int r = e / kVec, c = (e % kVec) * 4;
-    const int t = t0 + r;
-    float f[4] = {0.f, 0.f, 0.f, 0.f};
-    if (t < N) {
-      load4(x + ((size_t)bh * N + t) * D + c, f);
-      if (mean) {
+// Offsets, within one tile, of the 4-byte column `word` in rows r0 + k,
+// k = 0..7 (r0 a multiple of 8); row r0 + 8 j + k is at o[k] + 1024 j.
+SAGE_DEV void col_offsets(int word, int r0, uint32_t (&o)[8]) {
+  const int b = 4 * word;
+  const uint32_t base = (uint32_t)((b >> 7) * (kTok * kBoxBytes) + r0 * kBoxBytes + (b & 15));
+  const uint32_t c = (uint32_t)((b >> 4) & 7);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) f[i] = __fsub_rn(f[i], mean[bh * D + c + i]);
+  for (int k = 0; k < 8; ++k) o[k] = base + k * kBoxBytes + ((c ^ k) << 4);
+}
+
+// Shared-memory loads at 32-bit shared addresses (tile bytes land through
+// the async proxy; these follow the mbarrier waits that publish them).
+template <typename U>
+SAGE_DEV U lds(uint32_t addr);
+template <>
+SAGE_DEV uint32_t lds<uint32_t>(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+template <>
+SAGE_DEV float lds<float>(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+template <>
+SAGE_DEV uint4 lds<uint4>(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Calls f(r) for the rows r < rows of a tile, in order; FULL: rows == kTok.
+template <bool FULL, typename F>
+SAGE_DEV void each_row(int rows, F&& f) {
+#pragma unroll
+  for (int r = 0; r < kTok; ++r)
+    if (FULL || r < rows) f(r);
+}
+
+template <int D>
+struct QLayout {
+  static constexpr int W = D / 2;              // 32-bit words per token row
+  static constexpr int kTile = kTok * D * 2;   // bytes of one tensor tile
+  static constexpr int kItem = 3 * kTile;      // K, Q, V
+  static constexpr int kTiles = 2 * kItem;     // double buffer
+  static constexpr int kSlot = 3 * D * 4;      // k_mean, q_mean, v_mul of one buffer
+  static constexpr int kBytes = kTiles + 2 * kSlot;
+};
+
+enum Pass { kStatsPass = 0, kCodesPass = 1 };
+
+// One streaming pass over the 64-token chunks of all slices (chunk i of the
+// list is slice i / (Npad/64), block i % (Npad/64)); CTA c takes chunks
+// c, c + grid, ...  PASS selects the per-chunk work.
+template <typename T, int D, int PASS>
+__global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                 const __grid_constant__ CUtensorMap tm_k,
+                                                                 const __grid_constant__ CUtensorMap tm_v,
+                                                                 const QuantArgs a) {
+  using L = QLayout<D>;
+  using P = P16<T>;
+  constexpr int W = L::W;
+  extern __shared__ __align__(1024) uint8_t qsm[];
+  __shared__ __align__(8) uint64_t full[2], empty[2];
+  __shared__ int4 info[2];  // (item, bh, blk, -) per buffer; item -1: end
+  __shared__ int abort_s;
+  __shared__ uint2 mm[2][kCompute];  // K, Q: (max, min) pairs per (row group, word)
+  __shared__ float red[kComputeWarps];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nb = a.Npad / kTok;
+  const int nchunks = a.Npad / 64;
+  const size_t plane = (size_t)a.BH * nchunks * D;
+  // 1024-byte aligned start of the tiles (SWIZZLE_128B boxes)
+  uint8_t* const sm = qsm + ((1024u - (smem_u32(qsm) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(sm);
+
+  if (tid == 0) {
+    abort_s = 0;
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(&empty[0], kComputeWarps);
+    mbar_init(&empty[1], kComputeWarps);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kComputeWarps) {
+    // ------------------------------------------------------------- loader
+    if (lane != 0) return;
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    const bool need_q = PASS == kCodesPass || a.smooth_q;
+    for (int it = 0;; ++it) {
+      const int b = it & 1;
+      const int item = blockIdx.x + it * gridDim.x;
+      if (it >= 2 && !mbar_wait(&empty[b], ((it >> 1) - 1) & 1, &abort_s)) {
+        atomicCAS(a.err, 0, kErrTileWait);
+        abort_s = 1;
+        return;
+      }
+      if (item >= a.n_items) {
+        info[b] = make_int4(-1, 0, 0, 0);
+        mbar_arrive(&full[b]);
+        return;
+      }
+      const int bh = item / nb, blk = item % nb;
+      info[b] = make_int4(item, bh, blk, 0);
+      uint32_t bytes = (uint32_t)L::kTile * (need_q ? 3 : 2);
+      if (PASS == kCodesPass) bytes += (uint32_t)(D * 4) * (a.smooth_q ? 3 : 2);
+      mbar_arrive_expect_tx(&full[b], bytes);
+      uint8_t* dst = sm + b * L::kItem;
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x) {
+        const int off = x * kTok * kBoxBytes;
+        tma_load_3d(dst + off, &tm_k, &full[b], x * kBoxBytes, blk * kTok, bh);
+        if (need_q) tma_load_3d(dst + L::kTile + off, &tm_q, &full[b], x * kBoxBytes, blk * kTok, bh);
+        tma_load_3d(dst + 2 * L::kTile + off, &tm_v, &full[b], x * kBoxBytes, blk * kTok, bh);
+      }
+      if (PASS == kCodesPass) {
+        // the slice's means and V multipliers (written by the fold kernel)
+        float* sl = reinterpret_cast<float*>(sm + L::kTiles) + b * (3 * D);
+        bulk_load(sl, a.k_mean + (size_t)bh * D, D * 4, &full[b]);
+        if (a.smooth_q) bulk_load(sl + D, a.q_mean + (size_t)bh * D, D * 4, &full[b]);
+        bulk_load(sl + 2 * D, a.v_mul + (size_t)bh * D, D * 4, &full[b]);
       }
     }
-    const float fa = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
-    if (kNG == 1 || r < G) amax0 = fmaxf(amax0, fa);
-    else amax1 = fmaxf(amax1, fa);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) xs[r][c + i] = f[i];
   }
-  if (bias_mq && tid < D) smq[tid] = bias_mq[bh * D + tid];
-#pragma unroll
-  for (int g = 0; g < kNG; ++g) {
-    float a = g == 0 ? amax0 : amax1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if ((tid & 31) == 0) wmax[tid >> 5][g] = a;
-  }
-  __syncthreads();
-  if (tid < kNG) {
-    float a = 0.f;
-    for (int w = 0; w < 8; ++w) a = fmaxf(a, wmax[w][tid]);
-    const int gi = (t0 / G) + tid;
-    scale[(size_t)bh * (Npad / G) + gi] = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
-    ginv[tid] = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
-  }
-  __syncthreads();
-  // codes: each thread writes 4 consecutive codes per step
-  for (int e = tid; e < kRows * kVec; e += 256) {
-    const int r = e / kVec, c = (e % kVec) * 4;
-    const float inv = ginv[r / G];
-    uint32_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int qv = __float2int_rn(__fmul_rn(xs[r][c + i], inv));
-      qv = max(-127, min(127, qv));
-      packed |= ((uint32_t)(qv & 0xFF)) << (8 * i);
+
+  // --------------------------------------------------------------- compute
+  for (int it = 0;; ++it) {
+    const int b = it & 1;
+    const bool landed = mbar_wait(&full[b], (it >> 1) & 1, &abort_s);
+    if (!named_bar_and(kBarCompute, kCompute, landed)) {
+      if (tid == 0) {
+        atomicCAS(a.err, 0, kErrTileWait);
+        abort_s = 1;
+      }
+      return;
     }
-    *reinterpret_cast<uint32_t*>(codes + ((size_t)bh * Npad + t0 + r) * D + c) = packed;
-  }
-  if (bias_mq && tid < kRows) {
-    const int t = t0 + tid;
-    float acc = 0.f;
-    if (t < N)
-      for (int c = 0; c < D; ++c) acc = __fmaf_rn(smq[c], xs[tid][c], acc);
-    bias[(size_t)bh * Npad + t] = acc;
+    const int4 inf = info[b];
+    if (inf.x < 0) return;
+    const int bh = inf.y, blk = inf.z;
+    const int t0 = blk * kTok;
+    const int rows = min(kTok, a.N - t0);  // valid tokens (may be <= 0 in the padding)
+    const uint32_t tk = b * L::kItem, tq = tk + L::kTile, tv = tk + 2 * L::kTile;
+
+    if (PASS == kStatsPass) {
+      // Thread u < W: word u of the K rows, two sequential sums in token
+      // order; W <= u < 2W: the same for Q (smooth_q); 2W <= u < 3W: |V|
+      // maxima of word u - 2W (exact max / min of the raw values).
+      const int role = tid / W, word = tid % W;
+      if (role < 3 && (role != 1 || a.smooth_q)) {
+        uint32_t o[8];
+        col_offsets(word, 0, o);
+        float* p = a.part + role * plane + ((size_t)bh * nchunks + blk) * D + 2 * word;
+        if (role == 2) {
+          uint32_t mx = P::kNegInf, mn = P::kPosInf;
+          auto f = [&](int r) {
+            const uint32_t u = lds<uint32_t>(sb + tv + o[r & 7] + 1024 * (r >> 3));
+            mx = P::max(mx, u);
+            mn = P::min(mn, u);
+          };
+          if (rows == kTok)
+            each_row<true>(rows, f);
+          else
+            each_row<false>(rows, f);
+          float a0 = 0.f, a1 = 0.f;
+          if (rows > 0) {
+            float x0, x1, n0, n1;
+            unpack2<T>(mx, x0, x1);
+            unpack2<T>(mn, n0, n1);
+            a0 = fmaxf(fabsf(x0), fabsf(n0));
+            a1 = fmaxf(fabsf(x1), fabsf(n1));
+          }
+          *reinterpret_cast<float2*>(p) = make_float2(a0, a1);
+        } else {
+          const uint32_t src = role == 0 ? tk : tq;
+          uint64_t sum = f2pack(0.f, 0.f);
+          auto f = [&](int r) {
+            float lo, hi;
+            unpack2<T>(lds<uint32_t>(sb + src + o[r & 7] + 1024 * (r >> 3)), lo, hi);
+            sum = add2(sum, f2pack(lo, hi));
+          };
+          if (rows == kTok)
+            each_row<true>(rows, f);
+          else
+            each_row<false>(rows, f);
+          float s0, s1;
+          f2unpack(sum, s0, s1);
+          *reinterpret_cast<float2*>(p) = make_float2(s0, s1);
+        }
+      }
+    } else {
+        // shared addresses of this buffer's k_mean, q_mean, v_mul
+        const uint32_t kmean = sb + L::kTiles + 4 * (b * (3 * D));
+        const uint32_t qmean = kmean + 4 * D;
+        const uint32_t vmul = kmean + 8 * D;
+        constexpr int RG = kCompute / W;  // row groups: 4 (d=128) or 8 (d=64)
+        constexpr int RPG = kTok / RG;    // rows per group: 16 or 8
+        const int cw = tid % W, r0 = (tid / W) * RPG;  // this thread's column word and first row
+        uint32_t o[8];
+        col_offsets(cw, r0, o);
+        // A: per (row group, word) max and min of the raw K and Q values
+        {
+          uint32_t kx = P::kNegInf, kn = P::kPosInf, qx = P::kNegInf, qn = P::kPosInf;
+#pragma unroll
+          for (int r = 0; r < RPG; ++r) {
+            if (rows == kTok || r0 + r < rows) {
+              const uint32_t off = o[r & 7] + 1024 * (r >> 3);
+              const uint32_t uk = lds<uint32_t>(sb + tk + off);
+              const uint32_t uq = lds<uint32_t>(sb + tq + off);
+              kx = P::max(kx, uk);
+              kn = P::min(kn, uk);
+              qx = P::max(qx, uq);
+              qn = P::min(qn, uq);
+            }
+          }
+          mm[0][tid] = make_uint2(kx, kn);
+          mm[1][tid] = make_uint2(qx, qn);
+        }
+        named_bar_sync(kBarCompute, kCompute);
+        // B: granule maxima of |x~|.  RN(x - mean) is monotone in x, so the
+        // largest |x~| of a channel is at its largest or smallest raw value.
+        if (tid < 3 * W) {
+          const bool isk = tid < W;
+          const int g = isk ? 0 : (tid - W) / W, word = tid % W;
+          const int rg0 = isk ? 0 : g * (RG / 2), nrg = isk ? RG : RG / 2;
+          uint32_t x = P::kNegInf, n = P::kPosInf;
+          for (int i = 0; i < nrg; ++i) {
+            const uint2 e = mm[isk ? 0 : 1][(rg0 + i) * W + word];
+            x = P::max(x, e.x);
+            n = P::min(n, e.y);
+          }
+          float am = 0.f;
+          if ((isk ? rows : rows - 32 * g) > 0) {
+            float x0, x1, n0, n1;
+            unpack2<T>(x, x0, x1);
+            unpack2<T>(n, n0, n1);
+            if (isk || a.smooth_q) {
+              const uint32_t mean = isk ? kmean : qmean;
+              const float m0 = lds<float>(mean + 8 * word), m1 = lds<float>(mean + 8 * word + 4);
+              x0 = __fsub_rn(x0, m0);
+              n0 = __fsub_rn(n0, m0);
+              x1 = __fsub_rn(x1, m1);
+              n1 = __fsub_rn(n1, m1);
+            }
+            am = fmaxf(fmaxf(fabsf(x0), fabsf(n0)), fmaxf(fabsf(x1), fabsf(n1)));
+          }
+#pragma unroll
+          for (int s = 16; s > 0; s >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, s));
+          if (lane == 0) red[warp] = am;
+        }
+        named_bar_sync(kBarCompute, kCompute);
+        // C: scales, then codes.  K granule: warps [0, W/32); Q granule g:
+        // warps [W/32 (1 + g), W/32 (2 + g)).
+        constexpr int WPG = W / 32;
+        float mk = 0.f, mq0 = 0.f, mq1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < WPG; ++i) {
+          mk = fmaxf(mk, red[i]);
+          mq0 = fmaxf(mq0, red[WPG + i]);
+          mq1 = fmaxf(mq1, red[2 * WPG + i]);
+        }
+        if (tid == 0) a.k_scale[(size_t)bh * (a.Npad / 64) + t0 / 64] = mk > 0.f ? __fdiv_rn(mk, 127.0f) : 0.f;
+        if (tid == 1 || tid == 2) {
+          const float m = tid == 1 ? mq0 : mq1;
+          a.q_scale[(size_t)bh * (a.Npad / 32) + t0 / 32 + (tid - 1)] = m > 0.f ? __fdiv_rn(m, 127.0f) : 0.f;
+        }
+        const float ik = mk > 0.f ? __fdiv_rn(127.0f, mk) : 0.f;
+        const float iq0 = mq0 > 0.f ? __fdiv_rn(127.0f, mq0) : 0.f;
+        const float iq1 = mq1 > 0.f ? __fdiv_rn(127.0f, mq1) : 0.f;
+        {
+          // thread: 16-channel block cb of two adjacent rows' worth of lanes;
+          // each group of 8 lanes reads 8 distinct 16-byte bank groups
+          constexpr int CB = D / 16;
+          constexpr int RPT = kTok * CB / kCompute;  // rows per thread: 2 (d=128) or 1 (d=64)
+          const int cb = (tid & 3) + (CB == 8 ? 4 * ((tid >> 3) & 1) : 0);
+          const int rbase = (CB == 8 ? 2 * (tid >> 4) : 2 * (tid >> 3)) + ((tid >> 2) & 1);
+          const uint64_t rnd = f2pack(kRound, kRound);
+#pragma unroll 1
+          for (int which = 0; which < 2; ++which) {
+            const bool isk = which == 0;
+            const bool sub = isk || a.smooth_q;
+            const uint32_t src = isk ? tk : tq;
+            const uint32_t mean = isk ? kmean : qmean;
+            uint64_t negm[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              negm[j] = sub ? f2pack(-lds<float>(mean + 4 * (16 * cb + 2 * j)), -lds<float>(mean + 4 * (16 * cb + 2 * j + 1)))
+                            : f2pack(0.f, 0.f);
+            int8_t* dstc = isk ? a.k_codes : a.q_codes;
+#pragma unroll
+            for (int k = 0; k < RPT; ++k) {
+              const int row = rbase + 32 * k;
+              const float inv = isk ? ik : (row < 32 ? iq0 : iq1);
+              const uint4 h0 = lds<uint4>(sb + src + swz(row, 32 * cb));
+              const uint4 h1 = lds<uint4>(sb + src + swz(row, 32 * cb + 16));
+              const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+              float z[16];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                float lo, hi;
+                unpack2<T>(hw[j], lo, hi);
+                if (sub) f2unpack(add2(f2pack(lo, hi), negm[j]), lo, hi);
+                // scalar __fmul_rn: never merged into an fma with the add that
+                // follows, which would round x~ * inv and the integer rounding
+                // in one step (the packed multiply gets contracted)
+                lo = __fmul_rn(lo, inv);
+                hi = __fmul_rn(hi, inv);
+                f2unpack(add2(f2pack(lo, hi), rnd), z[2 * j], z[2 * j + 1]);
+              }
+              uint4 ov;
+              ov.x = low_bytes4(z[0], z[1], z[2], z[3]);
+              ov.y = low_bytes4(z[4], z[5], z[6], z[7]);
+              ov.z = low_bytes4(z[8], z[9], z[10], z[11]);
+              ov.w = low_bytes4(z[12], z[13], z[14], z[15]);
+              if (row >= rows) ov = make_uint4(0u, 0u, 0u, 0u);
+              *reinterpret_cast<uint4*>(dstc + ((size_t)bh * a.Npad + t0 + row) * D + 16 * cb) = ov;
+            }
+          }
+        }
+        if (a.smooth_q && tid < kTok) {
+          // Q-smoothing bias of token t0 + tid: fma chain over channels of
+          // mean_q[c] * k~[c] in channel order (k~ recomputed from the tile)
+          const int row = tid;
+          float acc = 0.f;
+          if (row < rows) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 8) {
+              const uint4 v4 = lds<uint4>(sb + tk + swz(row, 2 * c0));
+              const uint32_t uu[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float lo, hi;
+                unpack2<T>(uu[j], lo, hi);
+                const int c = c0 + 2 * j;
+                acc = __fmaf_rn(lds<float>(qmean + 4 * c), __fsub_rn(lo, lds<float>(kmean + 4 * c)), acc);
+                acc = __fmaf_rn(lds<float>(qmean + 4 * c + 4), __fsub_rn(hi, lds<float>(kmean + 4 * c + 4)), acc);
+              }
+            }
+          }
+          a.q_bias[(size_t)bh * a.Npad + t0 + row] = acc;
+        }
+        {
+          // V: thread = word cw (channels 2cw, 2cw+1) x rows r0 .. r0+RPG-1;
+          // e4m3 codes of v * (Vr / absmax_c), written transposed [c][t]
+          const float mul0 = lds<float>(vmul + 8 * cw), mul1 = lds<float>(vmul + 8 * cw + 4);
+          const uint64_t mul2v = f2pack(mul0, mul1);
+          uint32_t c0w[RPG / 4], c1w[RPG / 4];
+#pragma unroll
+          for (int r = 0; r < RPG; r += 4) {
+            float f0[4], f1[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float lo, hi;
+              unpack2<T>(lds<uint32_t>(sb + tv + o[(r + i) & 7] + 1024 * ((r + i) >> 3)), lo, hi);
+              f2unpack(mul2(f2pack(lo, hi), mul2v), f0[i], f1[i]);
+            }
+            uint32_t w0 = __byte_perm(e4m3x2(f0[0], f0[1]), e4m3x2(f0[2], f0[3]), 0x5410);
+            uint32_t w1 = __byte_perm(e4m3x2(f1[0], f1[1]), e4m3x2(f1[2], f1[3]), 0x5410);
+            if (rows < kTok) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (r0 + r + i >= rows) {
+                  w0 &= ~(0xFFu << (8 * i));
+                  w1 &= ~(0xFFu << (8 * i));
+                }
+            }
+            // a zero multiplier (all-zero channel) gives code 0, never -0
+            c0w[r / 4] = mul0 == 0.f ? 0u : w0;
+            c1w[r / 4] = mul1 == 0.f ? 0u : w1;
+          }
+          uint8_t* d0 = a.vt_codes + ((size_t)bh * D + 2 * cw) * a.Npad + t0 + r0;
+          uint8_t* d1 = d0 + a.Npad;
+          if constexpr (RPG == 16) {
+            *reinterpret_cast<uint4*>(d0) = make_uint4(c0w[0], c0w[1], c0w[2], c0w[3]);
+            *reinterpret_cast<uint4*>(d1) = make_uint4(c1w[0], c1w[1], c1w[2], c1w[3]);
+          } else {
+            *reinterpret_cast<uint2*>(d0) = make_uint2(c0w[0], c0w[1]);
+            *reinterpret_cast<uint2*>(d1) = make_uint2(c1w[0], c1w[1]);
+          }
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[b]);  // this warp is done with buffer b
   }
 }
 
-// ---------------------------------------------------------------- pass 3b
-// FP8 quantization of V, 128 tokens per block, written transposed:
-// grid (Npad/128, BH), 256 threads.
-template <typename T, int D>
-__global__ void __launch_bounds__(256) quant_v_fp8_kernel(const T* __restrict__ v, const float* __restrict__ v_mul,
-                                                          int N, int Npad, uint8_t* __restrict__ vt) {
-  constexpr int kTok = 128, kVec = D / 4;
-  __shared__ __align__(16) uint8_t tile[D][kTok + 16];
-  __shared__ float mul[D];
-  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int t0 = blk * kTok;
-  if (tid < D) mul[tid] = v_mul[bh * D + tid];
-  __syncthreads();
-  for (int e = tid; e < kTok * kVec; e += 256) {
-    const int r = e / kVec, c = (e % kVec) * 4;
-    const int t = t0 + r;
-    uint8_t cd[4] = {0, 0, 0, 0};
-    if (t < N) {
-      float f[4];
-      load4(v + ((size_t)bh * N + t) * D + c, f);
-      const uint16_t a = e4m3x2(__fmul_rn(f[0], mul[c]), __fmul_rn(f[1], mul[c + 1]));
-      const uint16_t b = e4m3x2(__fmul_rn(f[2], mul[c + 2]), __fmul_rn(f[3], mul[c + 3]));
-      cd[0] = (uint8_t)(a & 0xFF);
-      cd[1] = (uint8_t)(a >> 8);
-      cd[2] = (uint8_t)(b & 0xFF);
-      cd[3] = (uint8_t)(b >> 8);
-      // a zero multiplier (all-zero channel) gives code 0 as the oracle's rule
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (mul[c + i] == 0.f) cd[i] = 0;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) tile[c + i][r] = cd[i];
+// Per slice and tensor (blockIdx.y: 0 K sums, 1 |V| maxima, 2 Q sums), the
+// fold of the chunk partials in chunk order: thread c runs channel c's chain.
+// The partials stream through shared memory in pieces of kFoldRows chunks
+// (bulk copies into a double buffer), so every step of a chain reads shared
+// memory.
+template <int D>
+__global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
+  constexpr int kFoldRows = 4096 / D;  // 16 KB pieces
+  __shared__ __align__(16) float piece[2][kFoldRows * D];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int abort_s;
+  const int bh = blockIdx.x, c = threadIdx.x;
+  const int which = blockIdx.y == 0 ? 0 : blockIdx.y == 1 ? 2 : 1;  // part plane
+  const int nchunks = a.Npad / 64;
+  const int nvalid = (a.N + 63) / 64;
+  const float* src = a.part + (size_t)which * a.BH * nchunks * D + (size_t)bh * nchunks * D;
+  const int npieces = (nvalid + kFoldRows - 1) / kFoldRows;
+  if (c == 0) {
+    abort_s = 0;
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
   }
   __syncthreads();
-  for (int e = tid; e < D * (kTok / 16); e += 256) {
-    const int c = e / (kTok / 16), s = e % (kTok / 16);
-    const uint4 val = *reinterpret_cast<const uint4*>(&tile[c][s * 16]);
-    *reinterpret_cast<uint4*>(vt + ((size_t)bh * D + c) * Npad + t0 + s * 16) = val;
+  auto issue = [&](int p) {
+    const int rows = min(kFoldRows, nvalid - p * kFoldRows);
+    const uint32_t bytes = (uint32_t)rows * D * 4;
+    mbar_arrive_expect_tx(&bar[p & 1], bytes);
+    bulk_load(piece[p & 1], src + (size_t)p * kFoldRows * D, bytes, &bar[p & 1]);
+  };
+  if (c == 0) {
+    issue(0);
+    if (npieces > 1) issue(1);
+  }
+  float acc = 0.f;
+  bool ok = true;
+  for (int p = 0; p < npieces; ++p) {
+    if (!__syncthreads_and(mbar_wait(&bar[p & 1], (p >> 1) & 1, &abort_s))) {
+      ok = false;
+      break;
+    }
+    const int rows = min(kFoldRows, nvalid - p * kFoldRows);
+    const float* pc = piece[p & 1];
+    if (which == 2) {
+      for (int g = 0; g < rows; ++g) acc = fmaxf(acc, pc[g * D + c]);
+    } else {
+      for (int g = 0; g < rows; ++g) acc = __fadd_rn(acc, pc[g * D + c]);
+    }
+    __syncthreads();  // piece p & 1 is free
+    if (c == 0 && p + 2 < npieces) issue(p + 2);
+  }
+  if (!ok) {
+    if (c == 0) atomicCAS(a.err, 0, kErrTileWait);
+    return;
+  }
+  if (which == 0) {
+    a.k_mean[bh * D + c] = __fdiv_rn(acc, (float)a.N);
+  } else if (which == 1) {
+    a.q_mean[bh * D + c] = __fdiv_rn(acc, (float)a.N);
+  } else {
+    a.v_scale[bh * D + c] = acc > 0.f ? __fdiv_rn(acc, a.Vr) : 0.f;
+    a.v_mul[bh * D + c] = acc > 0.f ? __fdiv_rn(a.Vr, acc) : 0.f;
   }
 }
 
+// Per-device launch facts: SM count and resident CTAs per SM.
+struct LaunchFacts {
+  int sms = 0, per_sm = 0;
+};
+
+template <typename T, int D, int PASS>
+cudaError_t launch_facts(size_t smem, LaunchFacts* out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static LaunchFacts facts[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (facts[dev].sms == 0) {
+    e = cudaFuncSetAttribute(quant_pass_kernel<T, D, PASS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    LaunchFacts f;
+    e = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.per_sm, quant_pass_kernel<T, D, PASS>, kThreadsQ, smem);
+    if (e != cudaSuccess) return e;
+    if (f.per_sm < 1) return cudaErrorInvalidConfiguration;
+    facts[dev] = f;
+  }
+  *out = facts[dev];
+  return cudaSuccess;
+}
+
 template <typename T, int D>
-static cudaError_t quant_all(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
-                             const WsPtrs& w, cudaStream_t s) {
-  const T* qp = (const T*)q;
-  const T* kp = (const T*)k;
-  const T* vp = (const T*)v;
-  const int nchunks = pb.Npad / 64;
-  float* part = w.scratch;
-  float* v_mul = w.scratch + (size_t)3 * pb.BH * nchunks * D;
-  stats_partials_kernel<T, D><<<dim3(nchunks, pb.BH), D, 0, s>>>(kp, pb.smooth_q ? qp : nullptr, vp, pb.N,
-                                                                   nchunks, part);
-  stats_finalize_kernel<D><<<pb.BH, D, 0, s>>>(part, pb.N, nchunks, pb.smooth_q, Vr, w.k_mean, w.q_mean,
-                                               w.v_scale, v_mul);
-  quant_rows_int8_kernel<T, D, 32><<<dim3(nchunks, pb.BH), 256, 0, s>>>(
-      qp, pb.smooth_q ? w.q_mean : nullptr, pb.N, pb.Npad, w.q_codes, w.q_scale, nullptr, nullptr);
-  quant_rows_int8_kernel<T, D, 64><<<dim3(nchunks, pb.BH), 256, 0, s>>>(
-      kp, w.k_mean, pb.N, pb.Npad, w.k_codes, w.k_scale, pb.smooth_q ? w.q_mean : nullptr, w.q_bias);
-  quant_v_fp8_kernel<T, D><<<dim3(pb.Npad / 128, pb.BH), 256, 0, s>>>(vp, v_mul, pb.N, pb.Npad, w.vt_codes);
+cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem& pb, float Vr, const WsPtrs& w,
+                      cudaStream_t s) {
+  QuantArgs a;
+  a.q_codes = w.q_codes;
+  a.k_codes = w.k_codes;
+  a.vt_codes = w.vt_codes;
+  a.q_scale = w.q_scale;
+  a.k_scale = w.k_scale;
+  a.v_scale = w.v_scale;
+  a.k_mean = w.k_mean;
+  a.q_mean = w.q_mean;
+  a.q_bias = w.q_bias;
+  a.part = w.scratch;
+  a.v_mul = w.scratch + (size_t)3 * pb.BH * (pb.Npad / 64) * D;
+  a.err = w.error;
+  a.BH = pb.BH;
+  a.N = pb.N;
+  a.Npad = pb.Npad;
+  a.smooth_q = pb.smooth_q;
+  a.Vr = Vr;
+  a.n_items = pb.BH * (pb.Npad / kTok);
+
+  // 16-bit [BH][N][D] inputs seen as bytes: rows of 2D bytes, boxes of
+  // 128 bytes x 64 tokens (rows past N read as zero)
+  CUtensorMap tq, tk, tv;
+  const uint64_t row_bytes = (uint64_t)D * 2;
+  if (!make_tmap_u8_3d(&tq, q, row_bytes, pb.N, pb.BH, kBoxBytes, kTok) ||
+      !make_tmap_u8_3d(&tk, k, row_bytes, pb.N, pb.BH, kBoxBytes, kTok) ||
+      !make_tmap_u8_3d(&tv, v, row_bytes, pb.N, pb.BH, kBoxBytes, kTok))
+    return cudaErrorInvalidValue;
+
+  const size_t smem = QLayout<D>::kBytes + 1024;  // + alignment slack
+  LaunchFacts f0, f1;
+  cudaError_t e = launch_facts<T, D, kStatsPass>(smem, &f0);
+  if (e != cudaSuccess) return e;
+  e = launch_facts<T, D, kCodesPass>(smem, &f1);
+  if (e != cudaSuccess) return e;
+  const int g0 = (int)fmin((double)a.n_items, (double)f0.sms * f0.per_sm);
+  const int g1 = (int)fmin((double)a.n_items, (double)f1.sms * f1.per_sm);
+  quant_pass_kernel<T, D, kStatsPass><<<g0, kThreadsQ, smem, s>>>(tq, tk, tv, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  quant_fold_kernel<D><<<dim3(pb.BH, pb.smooth_q ? 3 : 2), D, 0, s>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  quant_pass_kernel<T, D, kCodesPass><<<g1, kThreadsQ, smem, s>>>(tq, tk, tv, a);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// Scratch floats the quantization pass needs (chunk partials, V multipliers).
+size_t quant_scratch_floats(int BH, int Npad, int d) {
+  return (size_t)3 * BH * (Npad / 64) * d + (size_t)BH * d;
 }
 
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
                                   const WsPtrs& w, cudaStream_t s) {
-  if (pb.dtype == 0) {
-    return pb.d == 128 ? quant_all<__half, 128>(q, k, v, pb, Vr, w, s) : quant_all<__half, 64>(q, k, v, pb, Vr, w, s);
-  }
-  return pb.d == 128 ? quant_all<__nv_bfloat16, 128>(q, k, v, pb, Vr, w, s)
-                     : quant_all<__nv_bfloat16, 64>(q, k, v, pb, Vr, w, s);
+  if (pb.dtype == 0)
+    return pb.d == 128 ? quant_run<__half, 128>(q, k, v, pb, Vr, w, s) : quant_run<__half, 64>(q, k, v, pb, Vr, w, s);
+  return pb.d == 128 ? quant_run<__nv_bfloat16, 128>(q, k, v, pb, Vr, w, s)
+                     : quant_run<__nv_bfloat16, 64>(q, k, v, pb, Vr, w, s);
 }
 
 }  // namespace sage

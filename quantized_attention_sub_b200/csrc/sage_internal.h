@@ -29,6 +29,10 @@ struct Problem {
   int BH, N, Npad, d, dtype, smooth_q, mode, causal;
 };
 
+// Floats of scratch the quantization pass needs: statistics partials
+// [3][BH][Npad/64][d] and V multipliers [BH][d].
+size_t quant_scratch_floats(int BH, int Npad, int d);
+
 // Smoothing statistics + INT8 Q/K + FP8 V (+ bias), enqueued on `s`.
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
                                   const WsPtrs& w, cudaStream_t s);
