@@ -473,8 +473,10 @@ ORC_EXPORT void orc_attn_int8_fp8(const int8_t* qc, const float* sq, const int8_
 /* ------------------------------------------------------------------------ */
 
 /* One block of 16 values x[0..15] (stride st) with global scale g:
- * bs = ue4m3(a_blk / (6 g)); code = e2m1(x / (g * dec(bs))); dec(bs) == 0 gives
- * codes 0.  Codes go to out[k] (one per byte, unpacked). */
+ * bs = ue4m3(a_blk / (6 g)); each value is scaled by the reciprocal of the
+ * block's decode factor, r = 1 / (g * dec(bs)) rounded once, and encoded:
+ * code = e2m1(x * r).  dec(bs) == 0 gives codes 0.  Codes go to out[k] (one
+ * per byte, unpacked). */
 static int fp4_block(const float* x, int st, float g, uint8_t* out)
 {
   float a = 0.0f;
@@ -483,8 +485,9 @@ static int fp4_block(const float* x, int st, float g, uint8_t* out)
   if (g > 0.0f) bs = orc_ue4m3_encode((double)(a / (6.0f * g)));
   float sd = (float)orc_ue4m3_decode(bs);
   float den = g * sd;
+  float r = (sd > 0.0f) ? 1.0f / den : 0.0f;
   for (int k = 0; k < 16; ++k)
-    out[k] = (uint8_t)((sd > 0.0f) ? orc_e2m1_encode((double)(x[k * st] / den)) : 0);
+    out[k] = (uint8_t)((sd > 0.0f) ? orc_e2m1_encode((double)(x[k * st] * r)) : 0);
   return bs;
 }
 
@@ -548,19 +551,23 @@ ORC_EXPORT void orc_quant_nvfp4_vt(const float* v, int BH, int N, int Npad, int 
   }
 }
 
-/* NVFP4 attention for one row.  S_ij = g_q g_k sum_c dq_ic dk_jc where the
+/* NVFP4 attention for one row.  x_ij = sum_c dq_ic dk_jc where the
  * dequantized values are code * dec(block scale) (exact products, summed in
- * double); then the same online softmax as the INT8 mode; P~ in NVFP4 along
- * keys with the constant global scale g_p = 1 / (6 * 448) (p <= 1); PV summed
- * exactly per tile and added in fp32; O = acc * g_p * g_v / l. */
+ * double, rounded once to fp32); then the logits and online softmax of the
+ * INT8 mode with kf = (g_q g_k) log2(e)/sqrt(d) in place of its per-granule
+ * factor and no P~ range factor; P~ in NVFP4 along keys with the constant
+ * global scale g_p = 1 / (6 * 448) (p <= 1); PV summed exactly per tile and
+ * added in fp32; O = acc * g_p * g_v / l. */
 static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq,
                            const uint8_t* kc, const uint8_t* ks, float gk,
                            const uint8_t* vc, const uint8_t* vs, float gv, const float* bias,
                            int N, int Npad, int d, int causal, double* qd, float* acc,
-                           float* tvals, float* pvals, uint8_t* pcodes, uint8_t* pbs, float* out_row)
+                           float* tvals, float* xvals, float* pvals, uint8_t* pcodes, uint8_t* pbs,
+                           float* out_row)
 {
   const float c_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   const float gp = 1.0f / (6.0f * 448.0f);
+  const float kf = (gq * gk) * c_log2;
   float m = -INFINITY, l = 0.0f;
   for (int c = 0; c < d; ++c) {
     acc[c] = 0.0f;
@@ -574,17 +581,23 @@ static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq
       double s = 0.0;
       for (int c = 0; c < d; ++c)
         s += qd[c] * orc_e2m1_decode(kc[(size_t)j * d + c]) * orc_ue4m3_decode(ks[(size_t)j * (d / 16) + c / 16]);
-      float t = (float)s * (gq * gk);
-      if (bias) t = t + bias[j];
-      t = t * c_log2;
+      const float x = (float)s;
+      const float t = bias ? fmaf(x, kf, bias[j] * c_log2) : x * kf;
+      xvals[j - j0] = x;
       tvals[j - j0] = t;
       if (t > mt) mt = t;
     }
-    float m_new = m > mt ? m : mt;
-    float alpha = orc_exp2(m - m_new);
+    const float m_new = m > mt ? m : mt;
+    const float alpha = orc_exp2(m - m_new);
+    /* d_j = t_j - m_new + 127 in one rounding, carried as g = d / 256 */
+    const float cs = (127.0f - m_new) * 0x1p-8f;
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
-      float p = (j0 + j > jmax) ? 0.0f : orc_exp2(tvals[j] - m_new);
+      float p = 0.0f;
+      if (j0 + j <= jmax) {
+        const float g = bias ? fmaf(tvals[j], 0x1p-8f, cs) : fmaf(xvals[j], kf * 0x1p-8f, cs);
+        p = exp2_g(sat01(g));
+      }
       pvals[j] = p;
       ps = ps + p;
     }
@@ -617,6 +630,7 @@ ORC_EXPORT void orc_attn_nvfp4(const uint8_t* qc, const uint8_t* qs, const float
     double* qd = (double*)malloc(sizeof(double) * d);
     float* acc = (float*)malloc(sizeof(float) * d);
     float* tv = (float*)malloc(sizeof(float) * 128);
+    float* xv = (float*)malloc(sizeof(float) * 128);
     float* pv = (float*)malloc(sizeof(float) * 128);
     uint8_t* pc = (uint8_t*)malloc(128);
     uint8_t pbs[8];
@@ -628,8 +642,8 @@ ORC_EXPORT void orc_attn_nvfp4(const uint8_t* qc, const uint8_t* qs, const float
                        kc + (size_t)bh * Npad * d, ks + (size_t)bh * Npad * (d / 16), gk[bh],
                        vc + (size_t)bh * d * Npad, vs + (size_t)bh * d * (Npad / 16), gv[bh],
                        bias ? bias + (size_t)bh * Npad : NULL, N, Npad, d, causal, qd, acc, tv,
-                       pv, pc, pbs, out + ((size_t)bh * nrows + r) * d);
+                       xv, pv, pc, pbs, out + ((size_t)bh * nrows + r) * d);
       }
-    free(qd); free(acc); free(tv); free(pv); free(pc);
+    free(qd); free(acc); free(tv); free(xv); free(pv); free(pc);
   }
 }
