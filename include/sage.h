@@ -76,10 +76,21 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype;
  *   q_bias   f32   [BH, Npad]      sum_c q_mean[c] * (k - k_mean)[n, c] (smooth_q)
  *   error    int32 (one word)      0, or the code of a wait that ran out
  *   scratch  f32                   partial sums of the statistics pass
- * In the NVFP4 mode q/k/vt_codes hold two e2m1 codes per byte (low nibble =
- * even index) with sizes halved along d (Q, K) or tokens (V^T); q/k/v_scale
- * hold ue4m3 block scales [BH,Npad,d/16], [BH,Npad,d/16], [BH,d,Npad/16];
- * global_scale holds fp32 [BH, 3] (Q, K, V). */
+ * In the NVFP4 mode (SageAttention3 abstract):
+ *   q_codes, k_codes  [BH, Npad, d/2]  two e2m1 codes per byte, low nibble =
+ *                     even channel; block of 16 channels per scale
+ *   vt_codes          [BH, d, Npad/2]  V^T, low nibble = even token; block of
+ *                     16 tokens per scale
+ *   q_scale, k_scale  ue4m3 block scales in 512-byte atoms, one atom per
+ *                     (128-row tile, 64 channels): atom index
+ *                     (bh * Npad/128 + row/128) * d/64 + channel/64, byte
+ *                     16*(r%32) + 4*(r/32) + b within it, r = row % 128,
+ *                     b = (channel % 64) / 16.  This is the layout the
+ *                     tensor cores read block scales in.
+ *   v_scale           the same atoms for V^T: index (bh * Npad/128 +
+ *                     token/128) * 2 + (token%128)/64, r = channel (rows
+ *                     d..127 of an atom are 0 when d = 64), b = (token%64)/16
+ *   global_scale      fp32 [BH, 4]: Q, K, V global scales (max |x| / 2688), 0 */
 typedef struct {
   size_t q_codes, k_codes, vt_codes, q_scale, k_scale, v_scale;
   size_t k_mean, q_mean, q_bias, global_scale, error, scratch;
@@ -117,7 +128,8 @@ SAGE_API sage_status sage_quantize_qkv(const void* q, const void* k, const void*
  *        the layout places before `scratch`), 1024-byte aligned; it receives
  *        the same codes, scales, means and bias as the workspace of
  *        sage_quantize_qkv, at the same offsets.
- *   Limit: 3*B*H*(Npad/64)*d + B*H*d words <= 4 Mi (16 MiB);
+ *   Limit: 3*B*H*(Npad/64)*d + B*H*d words (INT8/FP8 modes) or
+ *   7*B*H*(Npad/64)*d words (NVFP4) <= 4 Mi (16 MiB);
  *   larger problems return SAGE_ERR_UNSUPPORTED with the sizes in
  *   sage_last_error().
  *   The first call on a device looks up the array's device address once,

@@ -146,13 +146,28 @@ def alloc_workspace(B, H, N, d, mode, device="cuda") -> torch.Tensor:
 
 
 def ws_views(ws: torch.Tensor, B, H, N, d, mode) -> dict:
-    """Typed views of the quantized buffers inside a workspace (INT8/FP8 modes)."""
+    """Typed views of the quantized buffers inside a workspace.  NVFP4: packed
+    codes as bytes and the block scales as raw 512-byte atoms (the layout the
+    tensor cores read; include/sage.h gives the indexing)."""
     L = sage_workspace_layout(B, H, N, d, mode)
     BH, Np = B * H, (N + 127) // 128 * 128
 
     def view(off, nbytes, dtype, shape):
         return ws[off:off + nbytes].view(dtype).view(*shape)
 
+    if mode == MODE_NVFP4:
+        return dict(
+            q_codes=view(L.q_codes, BH * Np * d // 2, torch.uint8, (BH, Np, d // 2)),
+            k_codes=view(L.k_codes, BH * Np * d // 2, torch.uint8, (BH, Np, d // 2)),
+            vt_codes=view(L.vt_codes, BH * d * Np // 2, torch.uint8, (BH, d, Np // 2)),
+            q_sf_atoms=view(L.q_scale, BH * Np * d // 16, torch.uint8, (BH, Np // 128, d // 64, 512)),
+            k_sf_atoms=view(L.k_scale, BH * Np * d // 16, torch.uint8, (BH, Np // 128, d // 64, 512)),
+            v_sf_atoms=view(L.v_scale, BH * Np * 8, torch.uint8, (BH, Np // 128, 2, 512)),
+            global_scale=view(L.global_scale, BH * 16, torch.float32, (BH, 4)),
+            k_mean=view(L.k_mean, BH * d * 4, torch.float32, (BH, d)),
+            q_mean=view(L.q_mean, BH * d * 4, torch.float32, (BH, d)),
+            q_bias=view(L.q_bias, BH * Np * 4, torch.float32, (BH, Np)),
+        )
     return dict(
         q_codes=view(L.q_codes, BH * Np * d, torch.int8, (BH, Np, d)),
         k_codes=view(L.k_codes, BH * Np * d, torch.int8, (BH, Np, d)),

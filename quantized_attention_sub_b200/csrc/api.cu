@@ -51,8 +51,8 @@ sage_ws_layout layout_of(int B, int H, int N, int d, int mode) {
     L.vt_codes = take(BH * d * Np / 2);
     L.q_scale = take(BH * Np * d / 16);
     L.k_scale = take(BH * Np * d / 16);
-    L.v_scale = take(BH * d * Np / 16);
-    L.global_scale = take(BH * 3 * sizeof(float));
+    L.v_scale = take(BH * Np * 8);  // two 128-channel scale atoms per 128 tokens
+    L.global_scale = take(BH * 4 * sizeof(float));
   } else {
     L.q_codes = take(BH * Np * d);
     L.k_codes = take(BH * Np * d);
@@ -66,7 +66,7 @@ sage_ws_layout layout_of(int B, int H, int N, int d, int mode) {
   L.q_mean = take(BH * d * sizeof(float));
   L.q_bias = take(BH * Np * sizeof(float));
   // statistics partials and V multipliers of the quantize pass
-  L.scratch = take(sage::quant_scratch_floats((int)BH, (int)Np, d) * sizeof(float));
+  L.scratch = take(sage::quant_scratch_floats((int)BH, (int)Np, d, mode) * sizeof(float));
   L.total = off;
   return L;
 }
@@ -166,7 +166,6 @@ sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int d
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
   if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
     return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
-  if (mode == SAGE_MODE_NVFP4) return set_err(SAGE_ERR_UNSUPPORTED, "NVFP4 mode not built in this library%s");
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
   if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, 0};
@@ -186,14 +185,13 @@ sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
   if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
     return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
-  if (mode == SAGE_MODE_NVFP4) return set_err(SAGE_ERR_UNSUPPORTED, "NVFP4 mode not built in this library%s");
   if (!out) return set_err(SAGE_ERR_INVALID_ARG, "output buffer pointer is null%s");
   if (((uintptr_t)out) % kAlign) return set_err(SAGE_ERR_INVALID_ARG, "output buffer must be 1024-byte aligned%s");
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
   if (out_bytes < L.scratch)
     return set_err(SAGE_ERR_INVALID_ARG, "output buffer smaller than the layout's quantized region (layout.scratch)%s");
   const size_t Np = ((size_t)N + 127) / 128 * 128, BH = (size_t)B * H;
-  const size_t need = sage::quant_scratch_floats((int)BH, (int)Np, d);
+  const size_t need = sage::quant_scratch_floats((int)BH, (int)Np, d, mode);
   if (need > sage::static_scratch_floats()) {
     char buf[200];
     snprintf(buf, sizeof(buf), "problem needs %zu floats of static scratch; the maximum is %zu (16 MiB)", need,

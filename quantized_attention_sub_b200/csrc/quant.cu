@@ -78,8 +78,9 @@ struct QuantArgs {
   float* k_mean;
   float* q_mean;
   float* q_bias;
-  float* part;   // [3][BH][Npad/64][d]: K sums, Q sums, |V| maxima per 64-token chunk
-  float* v_mul;  // [BH][d]
+  float* part;   // [3 or 7][BH][Npad/64][d] per-chunk partials (see quant_scratch_floats)
+  float* v_mul;  // [BH][d] (INT8/FP8 modes)
+  float* gscale; // [BH][4] NVFP4 global scales (Q, K, V, 0)
   int* err;
   int BH, N, Npad, smooth_q, n_items;
   float Vr;
@@ -195,7 +196,7 @@ enum Pass { kStatsPass = 0, kCodesPass = 1 };
 // One streaming pass over the 64-token chunks of all slices (chunk i of the
 // list is slice i / (Npad/64), block i % (Npad/64)); CTA c takes chunks
 // c, c + grid, ...  PASS selects the per-chunk work.
-template <typename T, int D, int PASS>
+template <typename T, int D, int PASS, bool FP4>
 __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                  const __grid_constant__ CUtensorMap tm_k,
                                                                  const __grid_constant__ CUtensorMap tm_v,
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    const bool need_q = PASS == kCodesPass || a.smooth_q;
+    const bool need_q = PASS == kCodesPass || a.smooth_q || FP4;
     for (int it = 0;; ++it) {
       const int b = it & 1;
       const int item = blockIdx.x + it * gridDim.x;
@@ -250,7 +251,8 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
       const int bh = item / nb, blk = item % nb;
       info[b] = make_int4(item, bh, blk, 0);
       uint32_t bytes = (uint32_t)L::kTile * (need_q ? 3 : 2);
-      if (PASS == kCodesPass) bytes += (uint32_t)(D * 4) * (a.smooth_q ? 3 : 2);
+      if (PASS == kCodesPass) bytes += FP4 ? (uint32_t)(D * 4) * (a.smooth_q ? 2 : 1) + 16u
+                                           : (uint32_t)(D * 4) * (a.smooth_q ? 3 : 2);
       mbar_arrive_expect_tx(&full[b], bytes);
       uint8_t* dst = sm + b * L::kItem;
 #pragma unroll
@@ -265,7 +267,10 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
         float* sl = reinterpret_cast<float*>(sm + L::kTiles) + b * (3 * D);
         bulk_load(sl, a.k_mean + (size_t)bh * D, D * 4, &full[b]);
         if (a.smooth_q) bulk_load(sl + D, a.q_mean + (size_t)bh * D, D * 4, &full[b]);
-        bulk_load(sl + 2 * D, a.v_mul + (size_t)bh * D, D * 4, &full[b]);
+        if (FP4)
+          bulk_load(sl + 2 * D, a.gscale + (size_t)bh * 4, 16, &full[b]);
+        else
+          bulk_load(sl + 2 * D, a.v_mul + (size_t)bh * D, D * 4, &full[b]);
       }
     }
   }
@@ -288,7 +293,52 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
     const int rows = min(kTok, a.N - t0);  // valid tokens (may be <= 0 in the padding)
     const uint32_t tk = b * L::kItem, tq = tk + L::kTile, tv = tk + 2 * L::kTile;
 
-    if (PASS == kStatsPass) {
+    if (PASS == kStatsPass && FP4) {
+      // Thread u < W: word u of the K rows: two sequential sums in token order
+      // and the raw maxima and minima; W <= u < 2W: the same for Q (the sums
+      // only with smooth_q); 2W <= u < 3W: |V| maxima of word u - 2W.
+      const int role = tid / W, word = tid % W;
+      if (role < 3) {
+        uint32_t o[8];
+        col_offsets(word, 0, o);
+        const size_t cell = ((size_t)bh * nchunks + blk) * D + 2 * word;
+        const uint32_t src = role == 0 ? tk : role == 1 ? tq : tv;
+        const bool want_sum = role == 0 || (role == 1 && a.smooth_q);
+        uint32_t mx = P::kNegInf, mn = P::kPosInf;
+        uint64_t sum = f2pack(0.f, 0.f);
+        auto f = [&](int r) {
+          const uint32_t u = lds<uint32_t>(sb + src + o[r & 7] + 1024 * (r >> 3));
+          mx = P::max(mx, u);
+          mn = P::min(mn, u);
+          if (want_sum) {
+            float lo, hi;
+            unpack2<T>(u, lo, hi);
+            sum = add2(sum, f2pack(lo, hi));
+          }
+        };
+        if (rows == kTok)
+          each_row<true>(rows, f);
+        else
+          each_row<false>(rows, f);
+        float x0 = 0.f, x1 = 0.f, n0 = 0.f, n1 = 0.f;
+        if (rows > 0) {
+          unpack2<T>(mx, x0, x1);
+          unpack2<T>(mn, n0, n1);
+        }
+        if (role == 2) {
+          *reinterpret_cast<float2*>(a.part + 2 * plane + cell) =
+              make_float2(fmaxf(fabsf(x0), fabsf(n0)), fmaxf(fabsf(x1), fabsf(n1)));
+        } else {
+          if (want_sum) {
+            float s0, s1;
+            f2unpack(sum, s0, s1);
+            *reinterpret_cast<float2*>(a.part + role * plane + cell) = make_float2(s0, s1);
+          }
+          *reinterpret_cast<float2*>(a.part + (3 + 2 * role) * plane + cell) = make_float2(x0, x1);
+          *reinterpret_cast<float2*>(a.part + (4 + 2 * role) * plane + cell) = make_float2(n0, n1);
+        }
+      }
+    } else if (PASS == kStatsPass) {
       // Thread u < W: word u of the K rows, two sequential sums in token
       // order; W <= u < 2W: the same for Q (smooth_q); 2W <= u < 3W: |V|
       // maxima of word u - 2W (exact max / min of the raw values).
@@ -332,6 +382,136 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
           float s0, s1;
           f2unpack(sum, s0, s1);
           *reinterpret_cast<float2*>(p) = make_float2(s0, s1);
+        }
+      }
+    } else if (FP4) {
+      // NVFP4 codes: Q and K rows in blocks of 16 channels, V^T in blocks of
+      // 16 tokens per channel; per block a = max |x|, bs = ue4m3(a / (6 g)),
+      // r = 1 / (g * dec(bs)), code = e2m1(x * r), all IEEE fp32 steps.
+      const uint32_t kmean = sb + L::kTiles + 4 * (b * (3 * D));
+      const uint32_t qmean = kmean + 4 * D;
+      const uint32_t gsa = kmean + 8 * D;  // g_q, g_k, g_v, 0
+      const int tiles_per_slice = a.Npad / 128;
+      {
+        constexpr int CB = D / 16;
+        constexpr int RPT = kTok * CB / kCompute;  // rows per thread: 2 (d=128) or 1 (d=64)
+        const int cb = (tid & 3) + (CB == 8 ? 4 * ((tid >> 3) & 1) : 0);
+        const int rbase = (CB == 8 ? 2 * (tid >> 4) : 2 * (tid >> 3)) + ((tid >> 2) & 1);
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+          const bool isk = which == 0;
+          const bool sub = isk || a.smooth_q;
+          const uint32_t src = isk ? tk : tq;
+          const uint32_t mean = isk ? kmean : qmean;
+          const float g = lds<float>(gsa + (isk ? 4 : 0));
+          const float six_g = __fmul_rn(6.0f, g);
+          uint64_t negm[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            negm[j] = sub ? f2pack(-lds<float>(mean + 4 * (16 * cb + 2 * j)), -lds<float>(mean + 4 * (16 * cb + 2 * j + 1)))
+                          : f2pack(0.f, 0.f);
+          uint8_t* codes = reinterpret_cast<uint8_t*>(isk ? a.k_codes : a.q_codes);
+          uint8_t* sf = reinterpret_cast<uint8_t*>(isk ? a.k_scale : a.q_scale);
+#pragma unroll
+          for (int k = 0; k < RPT; ++k) {
+            const int row = rbase + 32 * k;
+            const uint4 h0 = lds<uint4>(sb + src + swz(row, 32 * cb));
+            const uint4 h1 = lds<uint4>(sb + src + swz(row, 32 * cb + 16));
+            const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            float x[16];
+            float am = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float lo, hi;
+              unpack2<T>(hw[j], lo, hi);
+              if (sub) f2unpack(add2(f2pack(lo, hi), negm[j]), lo, hi);
+              x[2 * j] = lo;
+              x[2 * j + 1] = hi;
+              am = fmaxf(am, fmaxf(fabsf(lo), fabsf(hi)));
+            }
+            uint32_t bs = 0;
+            float r = 0.f;
+            if (g > 0.f) {
+              bs = e4m3x2(__fdiv_rn(am, six_g), 0.f) & 0xFFu;
+              const float sd = e4m3_to_f32(bs);
+              if (sd > 0.f) r = __fdiv_rn(1.0f, __fmul_rn(g, sd));
+            }
+            uint2 cw = make_uint2(0u, 0u);
+            if (r > 0.f && row < rows) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) x[j] = __fmul_rn(x[j], r);
+              cw.x = e2m1x8(x);
+              cw.y = e2m1x8(x + 8);
+            }
+            if (row >= rows) bs = 0;
+            const int t = t0 + row;
+            *reinterpret_cast<uint2*>(codes + ((size_t)bh * a.Npad + t) * (D / 2) + 8 * cb) = cw;
+            const int m = t % 128;
+            sf[(((size_t)bh * tiles_per_slice + t / 128) * (D / 64) + cb / 4) * 512 + 16 * (m % 32) + 4 * (m / 32) +
+               (cb % 4)] = (uint8_t)bs;
+          }
+        }
+      }
+      if (a.smooth_q && tid < kTok) {
+        // Q-smoothing bias of token t0 + tid, as in the INT8/FP8 modes
+        const int row = tid;
+        float acc = 0.f;
+        if (row < rows) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 8) {
+            const uint4 v4 = lds<uint4>(sb + tk + swz(row, 2 * c0));
+            const uint32_t uu[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float lo, hi;
+              unpack2<T>(uu[j], lo, hi);
+              const int c = c0 + 2 * j;
+              acc = __fmaf_rn(lds<float>(qmean + 4 * c), __fsub_rn(lo, lds<float>(kmean + 4 * c)), acc);
+              acc = __fmaf_rn(lds<float>(qmean + 4 * c + 4), __fsub_rn(hi, lds<float>(kmean + 4 * c + 4)), acc);
+            }
+          }
+        }
+        a.q_bias[(size_t)bh * a.Npad + t0 + row] = acc;
+      }
+      if (tid < 4 * W) {
+        // V^T: thread = word (channels 2w, 2w+1) x one block of 16 tokens;
+        // tokens past N read as 0 (TMA fill), like the zero padding they stand for
+        const int word = tid % W, vb = tid / W;
+        uint32_t ov[8];
+        col_offsets(word, 16 * vb, ov);
+        const float g = lds<float>(gsa + 8);
+        const float six_g = __fmul_rn(6.0f, g);
+        float v0[16], v1[16];
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          unpack2<T>(lds<uint32_t>(sb + tv + ov[r & 7] + 1024 * (r >> 3)), v0[r], v1[r]);
+          a0 = fmaxf(a0, fabsf(v0[r]));
+          a1 = fmaxf(a1, fabsf(v1[r]));
+        }
+        uint8_t* sfv = reinterpret_cast<uint8_t*>(a.v_scale);
+        const int tt = t0 / 128, ka = (t0 % 128) / 64;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          float* vv = ch == 0 ? v0 : v1;
+          const float am = ch == 0 ? a0 : a1;
+          const int c = 2 * word + ch;
+          uint32_t bs = 0;
+          float r = 0.f;
+          if (g > 0.f) {
+            bs = e4m3x2(__fdiv_rn(am, six_g), 0.f) & 0xFFu;
+            const float sd = e4m3_to_f32(bs);
+            if (sd > 0.f) r = __fdiv_rn(1.0f, __fmul_rn(g, sd));
+          }
+          uint2 cw = make_uint2(0u, 0u);
+          if (r > 0.f) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) vv[j] = __fmul_rn(vv[j], r);
+            cw.x = e2m1x8(vv);
+            cw.y = e2m1x8(vv + 8);
+          }
+          *reinterpret_cast<uint2*>(a.vt_codes + ((size_t)bh * D + c) * (a.Npad / 2) + (t0 + 16 * vb) / 2) = cw;
+          sfv[(((size_t)bh * tiles_per_slice + tt) * 2 + ka) * 512 + 16 * (c % 32) + 4 * (c / 32) + vb] = (uint8_t)bs;
         }
       }
     } else {
@@ -530,23 +710,67 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
   }
 }
 
-// Per slice and tensor (blockIdx.y: 0 K sums, 1 |V| maxima, 2 Q sums), the
-// fold of the chunk partials in chunk order: thread c runs channel c's chain.
-// The partials stream through shared memory in pieces of kFoldRows chunks
-// (bulk copies into a double buffer), so every step of a chain reads shared
-// memory.
+// Folding the chunk partials of one slice: thread c runs channel c's chain
+// over the valid chunks in chunk order.  The partials stream through shared
+// memory in 16 KB pieces (bulk copies into a double buffer), so every step of
+// a chain reads shared memory.  Pieces are numbered across calls: piece k
+// uses buffer k & 1 with barrier parity (k >> 1) & 1.
+template <int D>
+struct Folder {
+  static constexpr int kRows = 4096 / D;  // chunks per 16 KB piece
+  float (*piece)[kRows * D];
+  uint64_t* bar;
+  int* abort;
+  int k = 0;
+  enum Op { kSum, kMax, kMin };
+
+  SAGE_DEV void issue(const float* src, int nvalid, int p) {
+    const int rows = min(kRows, nvalid - p * kRows);
+    const uint32_t bytes = (uint32_t)rows * D * 4;
+    const int kb = (k + p) & 1;
+    mbar_arrive_expect_tx(&bar[kb], bytes);
+    bulk_load(piece[kb], src + (size_t)p * kRows * D, bytes, &bar[kb]);
+  }
+  // Returns false (every thread) if a piece did not land in time.
+  SAGE_DEV bool run(const float* src, int nvalid, Op op, float& acc) {
+    const int c = threadIdx.x;
+    const int npieces = (nvalid + kRows - 1) / kRows;
+    acc = op == kSum ? 0.f : op == kMax ? -INFINITY : INFINITY;
+    if (c == 0) {
+      issue(src, nvalid, 0);
+      if (npieces > 1) issue(src, nvalid, 1);
+    }
+    for (int p = 0; p < npieces; ++p) {
+      const int kk = k + p;
+      if (!__syncthreads_and(mbar_wait(&bar[kk & 1], (kk >> 1) & 1, abort))) return false;
+      const int rows = min(kRows, nvalid - p * kRows);
+      const float* pc = piece[kk & 1];
+      if (op == kSum) {
+        for (int g = 0; g < rows; ++g) acc = __fadd_rn(acc, pc[g * D + c]);
+      } else if (op == kMax) {
+        for (int g = 0; g < rows; ++g) acc = fmaxf(acc, pc[g * D + c]);
+      } else {
+        for (int g = 0; g < rows; ++g) acc = fminf(acc, pc[g * D + c]);
+      }
+      __syncthreads();  // buffer kk & 1 is free
+      if (c == 0 && p + 2 < npieces) issue(src, nvalid, p + 2);
+    }
+    k += npieces;
+    return true;
+  }
+};
+
+// INT8/FP8 modes.  Per slice and tensor (blockIdx.y: 0 K sums, 1 |V| maxima,
+// 2 Q sums): means, V scales and multipliers.
 template <int D>
 __global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
-  constexpr int kFoldRows = 4096 / D;  // 16 KB pieces
-  __shared__ __align__(16) float piece[2][kFoldRows * D];
+  __shared__ __align__(16) float piece[2][Folder<D>::kRows * D];
   __shared__ __align__(8) uint64_t bar[2];
   __shared__ int abort_s;
   const int bh = blockIdx.x, c = threadIdx.x;
   const int which = blockIdx.y == 0 ? 0 : blockIdx.y == 1 ? 2 : 1;  // part plane
   const int nchunks = a.Npad / 64;
   const int nvalid = (a.N + 63) / 64;
-  const float* src = a.part + (size_t)which * a.BH * nchunks * D + (size_t)bh * nchunks * D;
-  const int npieces = (nvalid + kFoldRows - 1) / kFoldRows;
   if (c == 0) {
     abort_s = 0;
     mbar_init(&bar[0], 1);
@@ -554,34 +778,10 @@ __global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int p) {
-    const int rows = min(kFoldRows, nvalid - p * kFoldRows);
-    const uint32_t bytes = (uint32_t)rows * D * 4;
-    mbar_arrive_expect_tx(&bar[p & 1], bytes);
-    bulk_load(piece[p & 1], src + (size_t)p * kFoldRows * D, bytes, &bar[p & 1]);
-  };
-  if (c == 0) {
-    issue(0);
-    if (npieces > 1) issue(1);
-  }
-  float acc = 0.f;
-  bool ok = true;
-  for (int p = 0; p < npieces; ++p) {
-    if (!__syncthreads_and(mbar_wait(&bar[p & 1], (p >> 1) & 1, &abort_s))) {
-      ok = false;
-      break;
-    }
-    const int rows = min(kFoldRows, nvalid - p * kFoldRows);
-    const float* pc = piece[p & 1];
-    if (which == 2) {
-      for (int g = 0; g < rows; ++g) acc = fmaxf(acc, pc[g * D + c]);
-    } else {
-      for (int g = 0; g < rows; ++g) acc = __fadd_rn(acc, pc[g * D + c]);
-    }
-    __syncthreads();  // piece p & 1 is free
-    if (c == 0 && p + 2 < npieces) issue(p + 2);
-  }
-  if (!ok) {
+  Folder<D> f{piece, bar, &abort_s};
+  const float* src = a.part + ((size_t)which * a.BH + bh) * nchunks * D;
+  float acc;
+  if (!f.run(src, nvalid, which == 2 ? Folder<D>::kMax : Folder<D>::kSum, acc)) {
     if (c == 0) atomicCAS(a.err, 0, kErrTileWait);
     return;
   }
@@ -595,12 +795,75 @@ __global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
   }
 }
 
+// NVFP4.  Per slice and tensor (blockIdx.y: 0 K, 1 V, 2 Q): the means (K;
+// Q with smooth_q) and the global scale g = A / (6 * 448), A = the slice's
+// max |x~| over valid tokens.  RN(x - mean) is monotone in x, so per channel
+// that maximum is the larger of |RN(max - mean)| and |RN(min - mean)|.
+template <int D>
+__global__ void __launch_bounds__(D) quant_fold_fp4_kernel(const QuantArgs a) {
+  __shared__ __align__(16) float piece[2][Folder<D>::kRows * D];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int abort_s;
+  __shared__ float red[D / 32];
+  const int bh = blockIdx.x, c = threadIdx.x, y = blockIdx.y;
+  const int nchunks = a.Npad / 64;
+  const int nvalid = (a.N + 63) / 64;
+  const size_t plane = (size_t)a.BH * nchunks * D;
+  if (c == 0) {
+    abort_s = 0;
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  Folder<D> f{piece, bar, &abort_s};
+  auto src = [&](int pl) { return a.part + pl * plane + (size_t)bh * nchunks * D; };
+  bool ok = true;
+  float am = 0.f;
+  if (y == 1) {
+    ok = f.run(src(2), nvalid, Folder<D>::kMax, am);
+  } else {
+    const int role = y == 0 ? 0 : 1;  // 0 K, 1 Q
+    const bool has_mean = role == 0 || a.smooth_q;
+    float mu = 0.f, mx, mn;
+    if (has_mean) {
+      float s;
+      ok = f.run(src(role), nvalid, Folder<D>::kSum, s);
+      mu = __fdiv_rn(s, (float)a.N);
+      if (ok) (role == 0 ? a.k_mean : a.q_mean)[bh * D + c] = mu;
+    }
+    ok = ok && f.run(src(3 + 2 * role), nvalid, Folder<D>::kMax, mx);
+    ok = ok && f.run(src(4 + 2 * role), nvalid, Folder<D>::kMin, mn);
+    if (ok) {
+      if (has_mean) {
+        mx = __fsub_rn(mx, mu);
+        mn = __fsub_rn(mn, mu);
+      }
+      am = fmaxf(fabsf(mx), fabsf(mn));
+    }
+  }
+  if (!ok) {
+    if (c == 0) atomicCAS(a.err, 0, kErrTileWait);
+    return;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((c & 31) == 0) red[c >> 5] = am;
+  __syncthreads();
+  if (c == 0) {
+    float A = 0.f;
+    for (int i = 0; i < D / 32; ++i) A = fmaxf(A, red[i]);
+    a.gscale[bh * 4 + (y == 0 ? 1 : y == 1 ? 2 : 0)] = __fdiv_rn(A, 2688.0f);
+    if (y == 0) a.gscale[bh * 4 + 3] = 0.f;
+  }
+}
+
 // Per-device launch facts: SM count and resident CTAs per SM.
 struct LaunchFacts {
   int sms = 0, per_sm = 0;
 };
 
-template <typename T, int D, int PASS>
+template <typename T, int D, int PASS, bool FP4>
 cudaError_t launch_facts(size_t smem, LaunchFacts* out) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
@@ -611,12 +874,12 @@ cudaError_t launch_facts(size_t smem, LaunchFacts* out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (facts[dev].sms == 0) {
-    e = cudaFuncSetAttribute(quant_pass_kernel<T, D, PASS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(quant_pass_kernel<T, D, PASS, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchFacts f;
     e = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.per_sm, quant_pass_kernel<T, D, PASS>, kThreadsQ, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.per_sm, quant_pass_kernel<T, D, PASS, FP4>, kThreadsQ, smem);
     if (e != cudaSuccess) return e;
     if (f.per_sm < 1) return cudaErrorInvalidConfiguration;
     facts[dev] = f;
@@ -625,7 +888,7 @@ cudaError_t launch_facts(size_t smem, LaunchFacts* out) {
   return cudaSuccess;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool FP4>
 cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem& pb, float Vr, const WsPtrs& w,
                       cudaStream_t s) {
   QuantArgs a;
@@ -640,6 +903,7 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
   a.q_bias = w.q_bias;
   a.part = w.scratch;
   a.v_mul = w.scratch + (size_t)3 * pb.BH * (pb.Npad / 64) * D;
+  a.gscale = w.global_scale;
   a.err = w.error;
   a.BH = pb.BH;
   a.N = pb.N;
@@ -659,33 +923,50 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
 
   const size_t smem = QLayout<D>::kBytes + 1024;  // + alignment slack
   LaunchFacts f0, f1;
-  cudaError_t e = launch_facts<T, D, kStatsPass>(smem, &f0);
+  cudaError_t e = launch_facts<T, D, kStatsPass, FP4>(smem, &f0);
   if (e != cudaSuccess) return e;
-  e = launch_facts<T, D, kCodesPass>(smem, &f1);
+  e = launch_facts<T, D, kCodesPass, FP4>(smem, &f1);
   if (e != cudaSuccess) return e;
   const int g0 = (int)fmin((double)a.n_items, (double)f0.sms * f0.per_sm);
   const int g1 = (int)fmin((double)a.n_items, (double)f1.sms * f1.per_sm);
-  quant_pass_kernel<T, D, kStatsPass><<<g0, kThreadsQ, smem, s>>>(tq, tk, tv, a);
+  if (FP4 && D == 64) {
+    // rows 64..127 of the V^T scale atoms are never written: keep them 0
+    e = cudaMemsetAsync(w.v_scale, 0, (size_t)pb.BH * pb.Npad * 8, s);
+    if (e != cudaSuccess) return e;
+  }
+  quant_pass_kernel<T, D, kStatsPass, FP4><<<g0, kThreadsQ, smem, s>>>(tq, tk, tv, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  quant_fold_kernel<D><<<dim3(pb.BH, pb.smooth_q ? 3 : 2), D, 0, s>>>(a);
+  if (FP4)
+    quant_fold_fp4_kernel<D><<<dim3(pb.BH, 3), D, 0, s>>>(a);
+  else
+    quant_fold_kernel<D><<<dim3(pb.BH, pb.smooth_q ? 3 : 2), D, 0, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  quant_pass_kernel<T, D, kCodesPass><<<g1, kThreadsQ, smem, s>>>(tq, tk, tv, a);
+  quant_pass_kernel<T, D, kCodesPass, FP4><<<g1, kThreadsQ, smem, s>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 // Scratch floats the quantization pass needs (chunk partials, V multipliers).
-size_t quant_scratch_floats(int BH, int Npad, int d) {
+size_t quant_scratch_floats(int BH, int Npad, int d, int mode) {
+  if (mode == 2) return (size_t)7 * BH * (Npad / 64) * d;
   return (size_t)3 * BH * (Npad / 64) * d + (size_t)BH * d;
 }
 
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
                                   const WsPtrs& w, cudaStream_t s) {
+  if (pb.mode == 2) {
+    if (pb.dtype == 0)
+      return pb.d == 128 ? quant_run<__half, 128, true>(q, k, v, pb, Vr, w, s)
+                         : quant_run<__half, 64, true>(q, k, v, pb, Vr, w, s);
+    return pb.d == 128 ? quant_run<__nv_bfloat16, 128, true>(q, k, v, pb, Vr, w, s)
+                       : quant_run<__nv_bfloat16, 64, true>(q, k, v, pb, Vr, w, s);
+  }
   if (pb.dtype == 0)
-    return pb.d == 128 ? quant_run<__half, 128>(q, k, v, pb, Vr, w, s) : quant_run<__half, 64>(q, k, v, pb, Vr, w, s);
-  return pb.d == 128 ? quant_run<__nv_bfloat16, 128>(q, k, v, pb, Vr, w, s)
-                     : quant_run<__nv_bfloat16, 64>(q, k, v, pb, Vr, w, s);
+    return pb.d == 128 ? quant_run<__half, 128, false>(q, k, v, pb, Vr, w, s)
+                       : quant_run<__half, 64, false>(q, k, v, pb, Vr, w, s);
+  return pb.d == 128 ? quant_run<__nv_bfloat16, 128, false>(q, k, v, pb, Vr, w, s)
+                     : quant_run<__nv_bfloat16, 64, false>(q, k, v, pb, Vr, w, s);
 }
 
 }  // namespace sage

@@ -29,9 +29,11 @@ struct Problem {
   int BH, N, Npad, d, dtype, smooth_q, mode, causal;
 };
 
-// Floats of scratch the quantization pass needs: statistics partials
-// [3][BH][Npad/64][d] and V multipliers [BH][d].
-size_t quant_scratch_floats(int BH, int Npad, int d);
+// Floats of scratch the quantization pass needs.  INT8/FP8 modes: statistics
+// partials [3][BH][Npad/64][d] (K sums, Q sums, |V| maxima) and V multipliers
+// [BH][d].  NVFP4: partials [7][BH][Npad/64][d] (the same three planes, then
+// K maxima, K minima, Q maxima, Q minima of the raw values).
+size_t quant_scratch_floats(int BH, int Npad, int d, int mode);
 
 // Smoothing statistics + INT8 Q/K + FP8 V (+ bias), enqueued on `s`.
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,

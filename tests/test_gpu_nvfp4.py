@@ -1,0 +1,122 @@
+"""GPU parity of the NVFP4 mode (SageAttention3 abstract: microscaling FP4):
+the CUDA quantizers through the C ABI against the CPU oracle, bit for bit on
+codes, block scales, global scales, means and bias."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from quantized_attention_sub_b200 import api, inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_attention_sub_b200 import build
+    build.build()
+    api.lib()
+
+
+def unpack_nibbles(b):
+    """[..., n] bytes -> [..., 2n] e2m1 codes, low nibble first."""
+    b = np.asarray(b, np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def atoms_to_rows(atoms):
+    """Q/K scale atoms [BH, Npad/128, d/64, 512] -> [BH, Npad, d/16]."""
+    BH, T, KA, _ = atoms.shape
+    m = np.arange(128)
+    out = np.empty((BH, T * 128, KA * 4), np.uint8)
+    for ka in range(KA):
+        for kb in range(4):
+            out[:, :, ka * 4 + kb] = atoms[:, :, ka, 16 * (m % 32) + 4 * (m // 32) + kb].reshape(BH, T * 128)
+    return out
+
+
+def atoms_to_vt(atoms, d):
+    """V^T scale atoms [BH, Npad/128, 2, 512] -> [BH, d, Npad/16]; also the
+    unused rows (channels d..127), which must be 0."""
+    BH, T, _, _ = atoms.shape
+    c = np.arange(128)
+    full = np.empty((BH, 128, T * 8), np.uint8)
+    for t in range(T):
+        for ka in range(2):
+            for kb in range(4):
+                full[:, :, t * 8 + ka * 4 + kb] = atoms[:, t, ka, 16 * (c % 32) + 4 * (c // 32) + kb]
+    return full[:, :d], full[:, d:]
+
+
+def run_quant_fp4(q, k, v, smooth_q):
+    B, H, N, d = q.shape
+    ws = api.alloc_workspace(B, H, N, d, api.MODE_NVFP4)
+    api.sage_quantize_qkv(q, k, v, api.DTYPE_CODE[q.dtype], B, H, N, d, smooth_q, api.MODE_NVFP4, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    g = {n: t.cpu().numpy() for n, t in api.ws_views(ws, B, H, N, d, api.MODE_NVFP4).items()}
+    return ws, g
+
+
+def oracle_fp4(q, k, v, smooth_q):
+    B, H, N, d = q.shape
+    f = lambda t: t.float().cpu().reshape(B * H, N, d).numpy()
+    return orc.quantize_nvfp4(f(q), f(k), f(v), smooth_q)
+
+
+def assert_fp4_bitexact(g, o, d, smooth_q):
+    assert np.array_equal(unpack_nibbles(g["q_codes"]), o["q_codes"]), "q_codes"
+    assert np.array_equal(unpack_nibbles(g["k_codes"]), o["k_codes"]), "k_codes"
+    assert np.array_equal(unpack_nibbles(g["vt_codes"]), o["vt_codes"]), "vt_codes"
+    assert np.array_equal(atoms_to_rows(g["q_sf_atoms"]), o["q_bscale"]), "q block scales"
+    assert np.array_equal(atoms_to_rows(g["k_sf_atoms"]), o["k_bscale"]), "k block scales"
+    vbs, vpad = atoms_to_vt(g["v_sf_atoms"], d)
+    assert np.array_equal(vbs, o["vt_bscale"]), "v block scales"
+    assert not vpad.any(), "unused V scale rows must be 0"
+    gs = g["global_scale"]
+    for col, name in ((0, "q_gscale"), (1, "k_gscale"), (2, "v_gscale")):
+        assert np.array_equal(gs[:, col].view(np.uint32), o[name].view(np.uint32)), name
+    assert np.array_equal(g["k_mean"].view(np.uint32), o["k_mean"].view(np.uint32)), "k_mean"
+    if smooth_q:
+        assert np.array_equal(g["q_mean"].view(np.uint32), o["q_mean"].view(np.uint32)), "q_mean"
+        assert np.array_equal(g["q_bias"].view(np.uint32), o["q_bias"].view(np.uint32)), "q_bias"
+
+
+FP4_QUANT = [
+    # (N, d, dtype, law, smooth_q)
+    (128, 128, "bf16", "student_t3", False),
+    (1, 64, "fp16", "student_t3", False),
+    (77, 128, "fp16", "qk_bias", True),
+    (200, 64, "bf16", "k_bias_outlier", True),
+    (1000, 128, "bf16", "student_t3", False),
+]
+
+
+@pytest.mark.parametrize("N,d,dtype,law,smooth_q", FP4_QUANT)
+def test_nvfp4_quantize_bitexact(N, d, dtype, law, smooth_q):
+    w = inputs.variant(inputs.WORKLOADS["unit"], N=N, d=d, H=2, dtype=dtype, law=law, smooth_q=smooth_q,
+                       mode=api.MODE_NVFP4, seed=7000 + N + d)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    _, g = run_quant_fp4(q, k, v, smooth_q)
+    assert_fp4_bitexact(g, oracle_fp4(q, k, v, smooth_q), d, smooth_q)
+
+
+def test_nvfp4_quantize_edge_values():
+    """A zero V channel, an all-zero Q slice (global scale 0), a constant K
+    block, a value far above the rest (subnormal block scales elsewhere)."""
+    w = inputs.variant(inputs.WORKLOADS["unit"], N=150, d=64, H=2, dtype="fp16", law="student_t3",
+                       mode=api.MODE_NVFP4, seed=7777)
+    q, k, v = [t.clone() for t in inputs.generate(w)]
+    v[:, :, :, 3] = 0
+    q[:, 1] = 0
+    k[:, 0, 16:32, :] = 2.5
+    v[:, 0, 5, 7] = 3000.0
+    q, k, v = [t.cuda() for t in (q, k, v)]
+    for smooth_q in (False, True):
+        _, g = run_quant_fp4(q, k, v, smooth_q)
+        assert_fp4_bitexact(g, oracle_fp4(q, k, v, smooth_q), 64, smooth_q)
+    assert g["global_scale"][1, 0] == 0 and not unpack_nibbles(g["q_codes"][1]).any()
