@@ -164,6 +164,16 @@ SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, 
 SAGE_API sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,
                               int k_tile, int32_t* out, sage_stream_t stream);
 
+/* Parity helper of the NVFP4 mode (SageAttention3 abstract): one 128x128
+ * tile S[i][j] = sum_c (q_ic * sq_i,c/16) (k_jc * sk_j,c/16) of query tile
+ * q_tile and key tile k_tile of slice bh, computed from the workspace's
+ * packed e2m1 codes and ue4m3 block scales by the tensor-core path the
+ * NVFP4 attention uses (tcgen05.cp of the scale atoms into TMEM, tcgen05.mma
+ * kind::mxf4nvf4, FP32 accumulator); global scales are not applied.
+ * out: device float [128, 128], row = query.  NVFP4 workspace, d = 128. */
+SAGE_API sage_status sage_debug_fp4_s(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh,
+                                      int q_tile, int k_tile, float* out, sage_stream_t stream);
+
 /* Test helper for the failure path: launches one thread that waits on a
  * barrier nothing completes.  The bounded wait gives up after about 2 s, sets
  * the workspace error word, and the kernel returns; the CUDA context stays

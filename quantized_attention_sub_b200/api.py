@@ -21,7 +21,7 @@ DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
 
 EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_quantize_qkv_static",
             "sage_attn_quantized",
-            "sage_attn_fwd", "sage_debug_qk_s32", "sage_debug_timeout_probe", "sage_check", "sage_last_error")
+            "sage_attn_fwd", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_check", "sage_last_error")
 
 
 class WsLayout(ctypes.Structure):
@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.sage_attn_fwd.restype = i
         L.sage_debug_qk_s32.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
         L.sage_debug_qk_s32.restype = i
+        L.sage_debug_fp4_s.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
+        L.sage_debug_fp4_s.restype = i
         L.sage_debug_timeout_probe.argtypes = [vp, sz, vp]
         L.sage_debug_timeout_probe.restype = i
         L.sage_check.argtypes = [vp, sz, vp]
@@ -122,6 +124,10 @@ def sage_attn_fwd(q, k, v, out, B, H, N, d, causal, mode, dtype, smooth_q, ws, w
 
 def sage_debug_qk_s32(ws, ws_bytes, B, H, N, d, bh, q_tile, k_tile, out, stream=None):
     _raise(lib().sage_debug_qk_s32(_ptr(ws), ws_bytes, B, H, N, d, bh, q_tile, k_tile, _ptr(out), _stream(stream)))
+
+
+def sage_debug_fp4_s(ws, ws_bytes, B, H, N, d, bh, q_tile, k_tile, out, stream=None):
+    _raise(lib().sage_debug_fp4_s(_ptr(ws), ws_bytes, B, H, N, d, bh, q_tile, k_tile, _ptr(out), _stream(stream)))
 
 
 def sage_debug_timeout_probe(ws, ws_bytes, stream=None):

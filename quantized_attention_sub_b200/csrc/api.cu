@@ -252,6 +252,24 @@ sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int
                      "debug launch");
 }
 
+sage_status sage_debug_fp4_s(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,
+                             int k_tile, float* out, sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, SAGE_MODE_NVFP4);
+  if (st != SAGE_OK) return st;
+  if (d != 128) return set_err(SAGE_ERR_UNSUPPORTED, "the NVFP4 tensor-core path needs d = 128%s");
+  const int ntiles = (N + 127) / 128;
+  if (!out || bh < 0 || bh >= B * H || q_tile < 0 || q_tile >= ntiles || k_tile < 0 || k_tile >= ntiles)
+    return set_err(SAGE_ERR_INVALID_ARG, "debug tile out of range%s");
+  const sage_ws_layout L = layout_of(B, H, N, d, SAGE_MODE_NVFP4);
+  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  sage::Problem pb{B * H, N, ntiles * 128, d, 0, 0, SAGE_MODE_NVFP4, 0};
+  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_debug_fp4_s(resolve(const_cast<void*>(ws), L), pb, bh, q_tile, k_tile, out,
+                                              (cudaStream_t)stream),
+                     "debug launch");
+}
+
 sage_status sage_debug_timeout_probe(void* ws, size_t ws_bytes, sage_stream_t stream) {
   if (!ws || ws_bytes < sizeof(int) || ((uintptr_t)ws) % kAlign)
     return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null or misaligned%s");

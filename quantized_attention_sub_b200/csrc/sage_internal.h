@@ -52,6 +52,11 @@ cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, floa
 cudaError_t launch_debug_qk(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, int32_t* out,
                             cudaStream_t s);
 
+// One NVFP4 S tile (raw block-scaled dot products, FP32) through the
+// kind::mxf4nvf4 tensor-core path; d = 128.
+cudaError_t launch_debug_fp4_s(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, float* out,
+                               cudaStream_t s);
+
 // A kernel whose only wait can never complete: exercises the bounded-wait path.
 cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s);
 

@@ -229,6 +229,40 @@ SAGE_DEV uint64_t kmajor_desc(uint32_t smem_addr, int row_bytes) {
   return d;
 }
 
+// Shared-memory descriptor of one block-scale atom for tcgen05.cp: 32 rows of
+// 16 bytes, no swizzle (layout type 0), 8-row groups 128 bytes apart; the
+// leading offset is unused (one 16-byte core matrix per row).
+SAGE_DEV uint64_t sf_atom_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((128u >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
+}
+// Copy one block-scale atom (512 bytes) into TMEM columns [col, col + 4) of
+// every 32-lane quadrant (row m's four scales end up at lane m % 32 of each
+// quadrant, column col + m / 32).
+SAGE_DEV void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T: e2m1 operands with ue4m3
+// scales per 16 elements along K (K = 64 per instruction), FP32 accumulator;
+// the scales are read from TMEM at sfa / sfb.
+SAGE_DEV void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Instruction descriptor of the block-scaled FP4 MMA: a_format [7,10) and
+// b_format [10,13) = 1 (e2m1), scale format bit 23 = 0 (ue4m3), N>>3 at
+// [17,23), M>>4 at [24,29), scale-factor ids 0, K = 64 (bit 31 = 0).
+__host__ __device__ constexpr uint32_t idesc_fp4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor (kind::i8 / kind::f8f6f4, dense, K-major A and B).
 // c_format [4,6): 0 f16, 1 f32, 2 s32; a_format [7,10), b_format [10,13):
 // 1 = signed int8 for kind::i8, 0 = e4m3 for kind::f8f6f4; N>>3 at [17,23);

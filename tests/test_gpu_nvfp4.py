@@ -120,3 +120,33 @@ def test_nvfp4_quantize_edge_values():
         _, g = run_quant_fp4(q, k, v, smooth_q)
         assert_fp4_bitexact(g, oracle_fp4(q, k, v, smooth_q), 64, smooth_q)
     assert g["global_scale"][1, 0] == 0 and not unpack_nibbles(g["q_codes"][1]).any()
+
+
+def dequant_rows(codes, bscale):
+    """e2m1 codes [.., n] and ue4m3 scales [.., n/16] -> values (float64)."""
+    e2m1 = np.array([orc.e2m1_decode(c) for c in range(16)])
+    ue4m3 = np.array([orc.e4m3_decode(c & 0x7F) for c in range(256)])
+    return e2m1[codes] * np.repeat(ue4m3[bscale], 16, axis=-1)
+
+
+@pytest.mark.parametrize("N,law", [(256, "student_t3"), (300, "qk_bias")])
+def test_nvfp4_s_tile_tensor_core(N, law):
+    """One block-scaled S tile through tcgen05.cp + kind::mxf4nvf4 equals the
+    exact sum of products of the dequantized codes (FP32 accumulation)."""
+    w = inputs.variant(inputs.WORKLOADS["unit"], N=N, d=128, H=2, dtype="bf16", law=law, smooth_q=False,
+                       mode=api.MODE_NVFP4, seed=7100 + N)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    B, H, d = 1, 2, 128
+    ws, g = run_quant_fp4(q, k, v, False)
+    qd = dequant_rows(unpack_nibbles(g["q_codes"]), atoms_to_rows(g["q_sf_atoms"]))
+    kd = dequant_rows(unpack_nibbles(g["k_codes"]), atoms_to_rows(g["k_sf_atoms"]))
+    T = (N + 127) // 128
+    out = torch.empty(128, 128, dtype=torch.float32, device="cuda")
+    for bh in range(B * H):
+        for qt, kt in {(0, 0), (T - 1, 0), (0, T - 1), (T - 1, T - 1)}:
+            api.sage_debug_fp4_s(ws, ws.numel(), B, H, N, d, bh, qt, kt, out)
+            api.sage_check(ws, ws.numel())
+            ref = qd[bh, qt * 128:(qt + 1) * 128] @ kd[bh, kt * 128:(kt + 1) * 128].T
+            got = out.cpu().numpy().astype(np.float64)
+            scale = np.abs(ref).max() + 1e-30
+            assert np.abs(got - ref).max() <= 1e-5 * scale, (bh, qt, kt, np.abs(got - ref).max(), scale)
