@@ -214,12 +214,16 @@ sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int 
   if (!out) return set_err(SAGE_ERR_INVALID_ARG, "null output pointer%s");
   if (((uintptr_t)out) % 16) return set_err(SAGE_ERR_INVALID_ARG, "output must be 16-byte aligned%s");
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
-  if (mode == SAGE_MODE_NVFP4) return set_err(SAGE_ERR_UNSUPPORTED, "NVFP4 mode not built in this library%s");
+  if (mode == SAGE_MODE_NVFP4 && d != 128)
+    return set_err(SAGE_ERR_UNSUPPORTED, "the NVFP4 attention kernel needs d = 128%s");
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
   if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
   if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
+  if (mode == SAGE_MODE_NVFP4)
+    return cuda_status(sage::launch_attn_fp4(resolve(const_cast<void*>(ws), L), out, pb, (cudaStream_t)stream),
+                       "attention launch");
   // Pr: full e4m3 range with the FP32 accumulator, 224 with the FP16 one
   // (SageAttention2++ summary, Sec. 3.1)
   const float Pr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 224.0f : 448.0f;

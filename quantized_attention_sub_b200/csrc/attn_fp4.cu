@@ -12,8 +12,11 @@
 
 #include "sage_internal.h"
 #include "sage_ptx.cuh"
+#include "sage_softmax.cuh"
 
 namespace sage {
+
+using namespace sm;
 
 namespace {
 
@@ -96,7 +99,466 @@ __global__ void __launch_bounds__(128)
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+
+// ------------------------------------------------------------------ attention
+// One CTA owns one 128-query tile of one (b, h) slice (d = 128) and walks the
+// key tiles of 128 in order.  Warp roles (320 threads, 10 warps):
+//   warps 0-7   softmax: warpgroup h = warp / 4 handles key half h (keys
+//               [64h, 64h + 64) of every tile = one K = 64 MMA step);
+//               thread <-> row <-> TMEM lane
+//   warp 8      TMA producer (Q once, then a 3-stage ring of K and V^T tiles,
+//               each with its block-scale atoms); owns the TMEM allocation
+//   warp 9      MMA issuer (one thread): copies scale atoms into TMEM
+//               (tcgen05.cp), S = Q K^T and O += P~ V with kind::mxf4nvf4
+// TMEM (512 columns): S double buffer [0,128) and [128,256), O [256,384),
+// block scales from 384: Q, K per stage, V per stage, P~ per buffer.
+// Per key tile j, the two threads of row i (one per key half):
+//   load their 64 S values, take the half's logit max, exchange it,
+//   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
+//   p = exp2(t - m_new) (the method's exp2, the same argument steps as the
+//   INT8 mode), l_h = alpha l_h + sum p,
+//   per 16 keys: bs = ue4m3(max p / (6 g_p)), r = 1 / (g_p dec(bs)),
+//   P~ = e2m1(p r): 32 bytes of codes into the 64-byte swizzled P~ row and
+//   one 32-bit word of four scales into TMEM (tcgen05.st),
+//   wait for the previous P~V, multiply their half of the O row by alpha.
+// At the end l = l_0 + l_1 and O = acc * (g_p g_v) / l.
+// Every wait is bounded; a timeout records an error code in the workspace,
+// makes the other roles stop, and the CTA frees its TMEM.
+constexpr int kStagesF = 3;
+constexpr int kSoftmaxWarpsF = 8, kProducerWarpF = 8, kMmaWarpF = 9;
+constexpr int kThreadsF = 320;
+constexpr uint32_t kColO = 256, kColSfq = 384, kColSfk = 392, kColSfv = 416, kColSfp = 440;
+
+struct SmemF {
+  static constexpr int kTile = 128 * 64;  // 128 rows x 64 bytes (d = 128 or 128 keys of e2m1)
+  static constexpr int kSf = 1024;        // two scale atoms
+  static constexpr int off_q = 0;
+  static constexpr int off_sfq = off_q + kTile;
+  static constexpr int off_k = off_sfq + kSf;  // 1024-aligned
+  static constexpr int off_sfk = off_k + kStagesF * kTile;
+  static constexpr int off_v = off_sfk + kStagesF * kSf;
+  static constexpr int off_sfv = off_v + kStagesF * kTile;
+  static constexpr int off_p = off_sfv + kStagesF * kSf;  // [buffer 2]
+  static constexpr int off_bar = off_p + 2 * kTile;
+  static constexpr int off_x = off_bar + 256;  // [parity 2][half 2][row 128] floats
+  static constexpr int bytes = off_x + 2 * 2 * 128 * 4;
+  static constexpr int alloc = bytes + 1024;
+};
+static_assert(SmemF::off_k % 1024 == 0 && SmemF::off_v % 1024 == 0 && SmemF::off_p % 1024 == 0, "tile alignment");
+
+struct AttnF4Args {
+  const uint8_t* sfq;  // scale atoms, 1024 bytes per (slice, 128-row tile)
+  const uint8_t* sfk;
+  const uint8_t* sfv;
+  const float* gscale;  // [BH][4]
+  const float* bias;    // null unless smooth_q
+  void* out;
+  int* err;
+  int N, Npad, causal;
+  float c_log2;
+};
+
+enum : int { kErrProducerF = 0x311, kErrMmaF = 0x312, kErrSoftmaxF = 0x313, kErrDrainF = 0x314 };
+
+template <typename OutT, bool HAS_BIAS>
+__global__ void __launch_bounds__(kThreadsF, 1)
+    attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnF4Args a) {
+  using L = SmemF;
+  constexpr int D = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(smem + L::off_bar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kStagesF;
+  uint64_t* v_full = k_full + 2 * kStagesF;
+  uint64_t* v_empty = k_full + 3 * kStagesF;
+  uint64_t* s_full = k_full + 4 * kStagesF;  // [2]
+  uint64_t* s_free = s_full + 2;             // [2]
+  uint64_t* p_full = s_full + 4;             // [2]
+  uint64_t* o_done = s_full + 6;
+  uint64_t* x_bar = s_full + 7;  // [2 parities]
+  uint64_t* mma_fin = s_full + 9;
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 10);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* xch = (float*)(smem + L::off_x);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_ktiles = a.Npad / 128;
+  const int qt = a.causal ? (n_ktiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int bh = blockIdx.y;
+  const int T = a.causal ? qt + 1 : n_ktiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStagesF; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], kSoftmaxWarpsF);
+      mbar_init(&p_full[b], kSoftmaxWarpsF);
+      mbar_init(&x_bar[b], 256);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(mma_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarpF) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarpF) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const size_t tile0 = (size_t)bh * n_ktiles;  // scale atoms of this slice
+      mbar_arrive_expect_tx(q_full, L::kTile + L::kSf);
+      tma_load_3d(smem + L::off_q, &tm_q, q_full, 0, qt * 128, bh);
+      bulk_load(smem + L::off_sfq, a.sfq + (tile0 + qt) * L::kSf, L::kSf, q_full);
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < T; ++j) {
+        const int s = j % kStagesF, n = j / kStagesF;
+        if (j >= kStagesF && !mbar_wait(&k_empty[s], (n - 1) & 1, abort_flag)) {
+          fail(abort_flag, a.err, kErrProducerF);
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[s], L::kTile + L::kSf);
+        tma_load_3d(smem + L::off_k + s * L::kTile, &tm_k, &k_full[s], 0, j * 128, bh);
+        bulk_load(smem + L::off_sfk + s * L::kSf, a.sfk + (tile0 + j) * L::kSf, L::kSf, &k_full[s]);
+        issued_k = j + 1;
+        if (j >= kStagesF && !mbar_wait(&v_empty[s], (n - 1) & 1, abort_flag)) {
+          fail(abort_flag, a.err, kErrProducerF);
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[s], L::kTile + L::kSf);
+        tma_load_3d(smem + L::off_v + s * L::kTile, &tm_v, &v_full[s], j * 64, 0, bh);
+        bulk_load(smem + L::off_sfv + s * L::kSf, a.sfv + (tile0 + j) * L::kSf, L::kSf, &v_full[s]);
+        issued_v = j + 1;
+      }
+      // Drain: every load issued into shared memory must land before exit.
+      volatile int no_abort = 0;
+      if (!mbar_wait(q_full, 0, &no_abort)) atomicCAS(a.err, 0, kErrDrainF);
+      for (int j = max(0, issued_k - kStagesF); j < issued_k; ++j)
+        if (!mbar_wait(&k_full[j % kStagesF], (j / kStagesF) & 1, &no_abort)) atomicCAS(a.err, 0, kErrDrainF);
+      for (int j = max(0, issued_v - kStagesF); j < issued_v; ++j)
+        if (!mbar_wait(&v_full[j % kStagesF], (j / kStagesF) & 1, &no_abort)) atomicCAS(a.err, 0, kErrDrainF);
+    }
+  } else if (warp == kMmaWarpF) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_fp4(128, 128);
+      const uint32_t q_base = smem_u32(smem + L::off_q), k_base = smem_u32(smem + L::off_k);
+      const uint32_t v_base = smem_u32(smem + L::off_v), p_base = smem_u32(smem + L::off_p);
+      const uint32_t sfk_base = smem_u32(smem + L::off_sfk), sfv_base = smem_u32(smem + L::off_sfv);
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int ka = 0; ka < 2; ++ka)
+          tmem_cp_sf(tmem + kColSfq + 4 * ka, sf_atom_desc(smem_u32(smem + L::off_sfq) + 512 * ka));
+      }
+      auto issue_s = [&](int j) {
+        const int s = j % kStagesF;
+        const uint32_t kb = k_base + s * L::kTile, sfk = kColSfk + 8 * s;
+        for (int ka = 0; ka < 2; ++ka)
+          tmem_cp_sf(tmem + sfk + 4 * ka, sf_atom_desc(sfk_base + s * L::kSf + 512 * ka));
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_fp4(tmem + 128 * (j & 1), kmajor_desc(q_base + kk * 32, 64), kmajor_desc(kb + kk * 32, 64), idesc,
+                  tmem + kColSfq + 4 * kk, tmem + sfk + 4 * kk, kk > 0);
+        tc_commit(&s_full[j & 1]);
+      };
+      auto issue_pv = [&](int j) {
+        const int s = j % kStagesF;
+        const uint32_t pa = p_base + (j & 1) * L::kTile, vb = v_base + s * L::kTile, sfv = kColSfv + 8 * s;
+        for (int ka = 0; ka < 2; ++ka)
+          tmem_cp_sf(tmem + sfv + 4 * ka, sf_atom_desc(sfv_base + s * L::kSf + 512 * ka));
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_fp4(tmem + kColO, kmajor_desc(pa + kk * 32, 64), kmajor_desc(vb + kk * 32, 64), idesc,
+                  tmem + kColSfp + 8 * (j & 1) + 4 * kk, tmem + sfv + 4 * kk, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(o_done);
+      };
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        tc_commit(&k_empty[0]);
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) {
+          // S(j+1) into the buffer S(j-1) used, once the softmax has read it
+          const int s1 = (j + 1) % kStagesF;
+          if (!(ok = mbar_wait(&k_full[s1], ((j + 1) / kStagesF) & 1, abort_flag))) break;
+          if (j >= 1 && !(ok = mbar_wait(&s_free[(j + 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s(j + 1);
+          tc_commit(&k_empty[s1]);
+        }
+        if (!(ok = mbar_wait(&v_full[j % kStagesF], (j / kStagesF) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_pv(j);
+        tc_commit(&v_empty[j % kStagesF]);
+      }
+      if (!ok) fail(abort_flag, a.err, kErrMmaF);
+      // Every MMA issued so far must complete before the CTA frees TMEM.
+      tc_commit(mma_fin);
+      volatile int no_abort = 0;
+      if (!mbar_wait(mma_fin, 0, &no_abort)) atomicCAS(a.err, 0, kErrDrainF);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int h = warp >> 2, w4 = warp & 3;
+    const int r = threadIdx.x & 127;
+    const int row = qt * 128 + r;
+    const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
+    const uint32_t t_o = tmem + lane_off + kColO + h * 64;
+    uint8_t* prow0 = smem + L::off_p + r * 64;  // buffer 0; buffer 1 is kTile further
+    const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
+    const float4 gsc = *reinterpret_cast<const float4*>(a.gscale + (size_t)bh * 4);  // g_q, g_k, g_v, 0
+    const float kf = __fmul_rn(__fmul_rn(gsc.x, gsc.y), a.c_log2);
+    const float gp = __fdiv_rn(1.0f, 2688.0f);  // P~ global scale 1 / (6 * 448)
+    const float six_gp = __fmul_rn(6.0f, gp);
+    const int swz = (r >> 1) & 3;  // 64-byte swizzle of this row's 16-byte chunks
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int kbase = j * 128 + h * 64;
+      int lim = 64;
+      if (kbase + 63 >= a.N || (a.causal && j == qt)) {
+        lim = min(lim, a.N - kbase);
+        if (a.causal) lim = min(lim, row - kbase + 1);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[64];
+      const uint32_t t_s = tmem + lane_off + 128 * (j & 1) + h * 64;
+      tmem_ld32(t_s, sr);
+      tmem_ld32(t_s + 32, sr + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[j & 1]);
+
+      // t = x kf (or fma(x, kf, bias log2(e)/sqrt(d))), the INT8 mode's steps
+      if (lim < 64) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= lim) sr[c] = 0xFF800000u;
+      }
+      float mt;
+      if (!HAS_BIAS) {
+        float ga = -INFINITY, gb = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          ga = fmax3(ga, u2f(sr[c]), u2f(sr[c + 1]));
+          gb = fmax3(gb, u2f(sr[c + 2]), u2f(sr[c + 3]));
+        }
+        mt = __fmul_rn(fmaxf(ga, gb), kf);
+      } else {
+        const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
+        const float2 cl2 = make_float2(a.c_log2, a.c_log2);
+        float ma = -INFINITY, mb = -INFINITY;
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 bv = __ldg(b4 + c4);
+          const int c = 4 * c4;
+          const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
+                                       __fmul2_rn(make_float2(bv.x, bv.y), cl2));
+          const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf),
+                                       __fmul2_rn(make_float2(bv.z, bv.w), cl2));
+          sr[c] = f2u(ta.x);
+          sr[c + 1] = f2u(ta.y);
+          sr[c + 2] = f2u(tb.x);
+          sr[c + 3] = f2u(tb.y);
+          ma = fmax3(ma, ta.x, ta.y);
+          mb = fmax3(mb, tb.x, tb.y);
+        }
+        mt = fmaxf(ma, mb);
+      }
+      float* xs = xch + (j & 1) * 256;
+      xs[h * 128 + r] = mt;
+      mbar_arrive(&x_bar[j & 1]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&x_bar[j & 1], (j >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      mt = fmaxf(mt, xs[(h ^ 1) * 128 + r]);
+      const float m_new = fmaxf(m, mt);
+      const float alpha = exp2m(__fadd_rn(m, -m_new));
+      const float cs = __fmul_rn(__fadd_rn(127.0f, -m_new), 0x1p-8f);
+      const float gm = HAS_BIAS ? 0x1p-8f : __fmul_rn(kf, 0x1p-8f);
+
+      // p for the 64 keys, then per 16 keys the FP4 block: P~ codes into this
+      // tile's P buffer (last read by the P~V two tiles back, complete before
+      // the previous tile's rescale) and the four scales into TMEM
+      uint8_t* prow = prow0 + (j & 1) * L::kTile;
+      float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+      uint32_t cw[8];
+      uint32_t sfw = 0;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float p[16];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 16 * cc + 4 * e;
+          const float2 ga2 = make_float2(sat_fma(u2f(sr[c]), gm, cs), sat_fma(u2f(sr[c + 1]), gm, cs));
+          const float2 gb2 = make_float2(sat_fma(u2f(sr[c + 2]), gm, cs), sat_fma(u2f(sr[c + 3]), gm, cs));
+          const float2 pa = exp2g2(ga2), pb = exp2g2(gb2);
+          sa = __fadd2_rn(sa, pa);
+          sb = __fadd2_rn(sb, pb);
+          p[4 * e] = pa.x;
+          p[4 * e + 1] = pa.y;
+          p[4 * e + 2] = pb.x;
+          p[4 * e + 3] = pb.y;
+        }
+        float am = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) am = fmax3(am, p[e], p[e + 1]);
+        const uint32_t bs = e4m3x2(__fdiv_rn(am, six_gp), 0.f) & 0xFFu;
+        const float sd = e4m3_to_f32(bs);
+        const float rr = sd > 0.f ? __fdiv_rn(1.0f, __fmul_rn(gp, sd)) : 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) p[e] = __fmul_rn(p[e], rr);
+        cw[2 * cc] = e2m1x8(p);
+        cw[2 * cc + 1] = e2m1x8(p + 8);
+        sfw |= bs << (8 * cc);
+      }
+      *reinterpret_cast<uint4*>(prow + (((2 * h) ^ swz) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      *reinterpret_cast<uint4*>(prow + (((2 * h + 1) ^ swz) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      tmem_st1(tmem + lane_off + kColSfp + 8 * (j & 1) + 4 * h + w4, sfw);
+      fence_proxy_async_smem();
+      if (j > 0) {
+        // P~V of the previous tile must be done before its O rows are rescaled
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+          for (int i = 0; i < 2; ++i) {
+            uint32_t o[32];
+            tmem_ld32(t_o + 32 * i, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v2 = __fmul2_rn(make_float2(u2f(o[e]), u2f(o[e + 1])), make_float2(alpha, alpha));
+              o[e] = f2u(v2.x);
+              o[e + 1] = f2u(v2.y);
+            }
+            tmem_st32(t_o + 32 * i, o);
+          }
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[j & 1]);
+      l = __fadd_rn(__fmul_rn(alpha, l), (sa.x + sa.y) + (sb.x + sb.y));
+      m = m_new;
+    }
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(o_done, (T - 1) & 1, abort_flag))) ok = false;
+    if (ok) {
+      const int jx = T;
+      float* xs = xch + (jx & 1) * 256;
+      xs[h * 128 + r] = l;
+      mbar_arrive(&x_bar[jx & 1]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&x_bar[jx & 1], (jx >> 1) & 1, abort_flag))) ok = false;
+      else l = h == 0 ? __fadd_rn(l, xs[128 + r]) : __fadd_rn(xs[r], l);
+    }
+    if (!ok) {
+      fail(abort_flag, a.err, kErrSoftmaxF);
+    } else {
+      tc_fence_after();
+      const float gpv = __fmul_rn(gp, gsc.z);
+      OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D + h * 64;
+#pragma unroll 1
+      for (int i = 0; i < 2; ++i) {
+        uint32_t o[32];
+        tmem_ld32(t_o + 32 * i, o);
+        tmem_ld_wait();
+        if (row < a.N) {
+          uint32_t hh[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            hh[e] = pack2<OutT>(__fdiv_rn(__fmul_rn(u2f(o[2 * e]), gpv), l),
+                                __fdiv_rn(__fmul_rn(u2f(o[2 * e + 1]), gpv), l));
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            *reinterpret_cast<uint4*>(orow + 32 * i + 8 * v4) =
+                make_uint4(hh[4 * v4], hh[4 * v4 + 1], hh[4 * v4 + 2], hh[4 * v4 + 3]);
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kProducerWarpF) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <typename OutT, bool HAS_BIAS>
+cudaError_t run_attn_fp4(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnF4Args& a,
+                         int BH, int ntiles, cudaStream_t s) {
+  auto kern = attn_fp4_kernel<OutT, HAS_BIAS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemF::alloc);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(ntiles, BH), kThreadsF, SmemF::alloc, s>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_attn_fp4(const WsPtrs& w, void* out, const Problem& pb, cudaStream_t s) {
+  if (pb.d != 128) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv;
+  // packed codes: Q, K [BH][Npad][64 bytes]; V^T [BH][128][Npad/2 bytes]; boxes 64 bytes x 128 rows
+  if (!make_tmap_u8_3d(&mq, w.q_codes, 64, pb.Npad, pb.BH, 64, 128) ||
+      !make_tmap_u8_3d(&mk, w.k_codes, 64, pb.Npad, pb.BH, 64, 128) ||
+      !make_tmap_u8_3d(&mv, w.vt_codes, pb.Npad / 2, 128, pb.BH, 64, 128))
+    return cudaErrorInvalidValue;
+  AttnF4Args a;
+  a.sfq = reinterpret_cast<const uint8_t*>(w.q_scale);
+  a.sfk = reinterpret_cast<const uint8_t*>(w.k_scale);
+  a.sfv = reinterpret_cast<const uint8_t*>(w.v_scale);
+  a.gscale = w.global_scale;
+  a.bias = pb.smooth_q ? w.q_bias : nullptr;
+  a.out = out;
+  a.err = w.error;
+  a.N = pb.N;
+  a.Npad = pb.Npad;
+  a.causal = pb.causal;
+  a.c_log2 = (float)(1.4426950408889634 / sqrt((double)pb.d));
+  const int ntiles = pb.Npad / 128;
+  const bool bias = a.bias != nullptr;
+  if (pb.dtype == 0)
+    return bias ? run_attn_fp4<__half, true>(mq, mk, mv, a, pb.BH, ntiles, s)
+                : run_attn_fp4<__half, false>(mq, mk, mv, a, pb.BH, ntiles, s);
+  return bias ? run_attn_fp4<__nv_bfloat16, true>(mq, mk, mv, a, pb.BH, ntiles, s)
+              : run_attn_fp4<__nv_bfloat16, false>(mq, mk, mv, a, pb.BH, ntiles, s);
+}
 
 cudaError_t launch_debug_fp4_s(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, float* out,
                                cudaStream_t s) {

@@ -48,6 +48,9 @@ size_t static_scratch_floats();
 // Fused attention (FP32 PV accumulator).
 cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s);
 
+// Fused NVFP4 attention (kind::mxf4nvf4 for S and P~V, FP32 accumulator); d = 128.
+cudaError_t launch_attn_fp4(const WsPtrs& w, void* out, const Problem& pb, cudaStream_t s);
+
 // INT32 S tile through the tensor-core path.
 cudaError_t launch_debug_qk(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, int32_t* out,
                             cudaStream_t s);

@@ -150,3 +150,44 @@ def test_nvfp4_s_tile_tensor_core(N, law):
             got = out.cpu().numpy().astype(np.float64)
             scale = np.abs(ref).max() + 1e-30
             assert np.abs(got - ref).max() <= 1e-5 * scale, (bh, qt, kt, np.abs(got - ref).max(), scale)
+
+
+ATTN_FP4 = [
+    # (N, dtype, law, smooth_q, causal)
+    (128, "bf16", "student_t3", False, False),
+    (1, "bf16", "student_t3", False, False),
+    (33, "fp16", "k_bias", False, True),
+    (256, "bf16", "student_t3", False, False),
+    (300, "fp16", "qk_bias", True, True),
+    (1000, "bf16", "student_t3", False, True),
+    (640, "fp16", "k_bias_outlier", True, False),
+]
+
+
+@pytest.mark.parametrize("N,dtype,law,smooth_q,causal", ATTN_FP4)
+def test_nvfp4_attention_matches_oracle(N, dtype, law, smooth_q, causal):
+    """The fused kind::mxf4nvf4 attention against the oracle's NVFP4
+    attention on the same (bit-identical) codes and scales, output rounded to
+    the dtype, with the INT8/FP8 modes' bounds."""
+    from test_gpu_parity import compare_out, to_dtype_np
+    w = inputs.variant(inputs.WORKLOADS["unit"], N=N, d=128, H=2, dtype=dtype, law=law, smooth_q=smooth_q,
+                       mode=api.MODE_NVFP4, causal=causal, seed=7300 + N)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    B, H, d = 1, 2, 128
+    ws = api.alloc_workspace(B, H, N, d, api.MODE_NVFP4)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, causal, api.MODE_NVFP4, api.DTYPE_CODE[q.dtype], smooth_q, ws,
+                      ws.numel())
+    api.sage_check(ws, ws.numel())
+    ref = to_dtype_np(orc.attention_nvfp4(oracle_fp4(q, k, v, smooth_q), causal), dtype)
+    got = out.float().cpu().reshape(B * H, N, d).numpy()
+    compare_out(got, ref, dtype, (N, dtype, law, smooth_q, causal))
+
+
+def test_nvfp4_attention_rejects_d64():
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
+    ws = api.alloc_workspace(1, 1, 128, 64, api.MODE_NVFP4)
+    with pytest.raises(api.SageError) as e:
+        api.sage_attn_fwd(q, q, q, torch.empty_like(q), 1, 1, 128, 64, False, api.MODE_NVFP4, 1, False, ws,
+                          ws.numel())
+    assert e.value.status == api.SAGE_ERR_UNSUPPORTED
