@@ -39,6 +39,15 @@ from quantized_attention_sub_b200 import api, inputs  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio 4.5 / 2.25 PFLOP/s (INT8 dense equals FP8 dense)
+FP4_OVER_BF16 = 4.0   # nominal dense ratio 9 / 2.25 PFLOP/s
+
+# per mode: tensor peak ratio to bf16, attention kernel, arithmetic description
+MODE_INFO = {
+    0: (FP8_OVER_BF16, "attn_i8f8_kernel", "int8 QK / e4m3 PV, fp32 softmax and accumulation"),
+    1: (FP8_OVER_BF16, "attn_i8f8_kernel (FP16 accumulator)",
+        "int8 QK / e4m3 PV, fp16 PV accumulation per 64 keys, fp32 softmax"),
+    2: (FP4_OVER_BF16, "attn_fp4_kernel", "e2m1 QK and PV with ue4m3 block scales, fp32 softmax and accumulation"),
+}
 
 
 def load_peaks():
@@ -131,8 +140,12 @@ def oracle_sample(w, max_rows):
     f = lambda t: t.float().reshape(1, w.N, w.d).numpy()
     rows = np.unique(np.linspace(0, w.N - 1, min(max_rows, w.N)).astype(np.int32))
     t0 = time.perf_counter()
-    qz = orc.quantize_int8_fp8(f(q), f(k), f(v), smooth_q=w.smooth_q, mode=w.mode)
-    orc.attention_int8_fp8(qz, w.causal, rows=rows)
+    if w.mode == 2:
+        qz = orc.quantize_nvfp4(f(q), f(k), f(v), smooth_q=w.smooth_q)
+        orc.attention_nvfp4(qz, w.causal, rows=rows)
+    else:
+        qz = orc.quantize_int8_fp8(f(q), f(k), f(v), smooth_q=w.smooth_q, mode=w.mode)
+        orc.attention_int8_fp8(qz, w.causal, rows=rows)
     dt = time.perf_counter() - t0
     keys = (rows.astype(np.float64) + 1) if w.causal else np.full(len(rows), float(w.N))
     ops = float(4.0 * w.d * keys.sum())
@@ -157,7 +170,7 @@ def run_reference(args, w, ws, rank):
     line = {"impl": "reference", "metric": "attention TOPS (visible-pair count)", "value": value,
             "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8/fp8 codes, fp32 arithmetic", "data": "synthetic",
+            "vs_baseline": None, "dtype": MODE_INFO[w.mode][2] + " (CPU oracle)", "data": "synthetic",
             "config": config_of(w, args, ws),
             "cpu_baseline": {"value": value, "unit": "TOPS", "cores": thr, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -252,17 +265,19 @@ def main():
 
     # roofline of the dominant kernel (attention), live CUDA-event time
     peaks, peak_src = load_peaks()
-    peak_fp8 = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    ratio, kname, dtype_desc = MODE_INFO[w.mode]
+    peak_fp8 = peaks["bf16_tflops_sustained"] * ratio
     achieved = inputs.executed_ops(w) / (attn_avg * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "attn_i8f8_kernel", "achieved": achieved, "peak": peak_fp8,
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak_fp8,
                 "unit": "TFLOP/s", "frac": achieved / peak_fp8,
-                "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense FP8/INT8 : BF16 ratio)" % (
-                    peak_src, FP8_OVER_BF16),
+                "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense %s : BF16 ratio)" % (
+                    peak_src, ratio, "FP4" if w.mode == 2 else "FP8/INT8"),
                 "traffic": None, "attn_ms": attn_avg}
     # the quantization pass (HBM-bound): 16-bit Q, K, V read once, int8/e4m3
     # codes written, statistics and scales (small) not counted
     Np = (N + 127) // 128 * 128
-    q_bytes = 3 * B * H * N * d * 2 + 3 * B * H * Np * d
+    # NVFP4: half a byte of code plus 1/16 byte of block scale per element
+    q_bytes = 3 * B * H * N * d * 2 + (3 * B * H * Np * d * 9 // 16 if w.mode == 2 else 3 * B * H * Np * d)
     hbm = peaks["hbm_gbs"]
     quant_line = {"bound": "hbm", "kernel": "quant_pass_kernel (stats) + quant_fold_kernel + quant_pass_kernel (codes)", "ms": quant_avg,
                   "algorithmic_bytes": q_bytes, "achieved": q_bytes / (quant_avg * 1e-3) / 1e9,
@@ -299,7 +314,7 @@ def main():
     line = {"metric": "attention TOPS (4*B*H*d per visible (query,key) pair / time)", "value": value,
             "unit": "TOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8 QK / e4m3 PV, fp32 softmax and accumulation", "data": "synthetic",
+            "dtype": dtype_desc, "data": "synthetic",
             "config": config_of(w, args, ws),
             "value_square_count": ops_square / (ms * 1e-3) / 1e12,
             "roofline": roofline,

@@ -191,3 +191,26 @@ def test_nvfp4_attention_rejects_d64():
         api.sage_attn_fwd(q, q, q, torch.empty_like(q), 1, 1, 128, 64, False, api.MODE_NVFP4, 1, False, ws,
                           ws.numel())
     assert e.value.status == api.SAGE_ERR_UNSUPPORTED
+
+
+def test_full_size_nvfp4_sampled_rows():
+    """The B1 H16 N16384 d128 bf16 NVFP4 workload at full size, in the launch
+    configuration the bench times: quantization bit-exact everywhere, the
+    output on sampled rows per head (first, tile edges, last, random)."""
+    from test_gpu_parity import compare_out, to_dtype_np
+    w = inputs.WORKLOADS["nvfp4"]
+    B, H, N, d = w.shape()
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    ws = api.alloc_workspace(B, H, N, d, api.MODE_NVFP4)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, w.causal, api.MODE_NVFP4, api.DTYPE_CODE[q.dtype], w.smooth_q,
+                      ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    g = {n: t.cpu().numpy() for n, t in api.ws_views(ws, B, H, N, d, api.MODE_NVFP4).items()}
+    oz = oracle_fp4(q, k, v, w.smooth_q)
+    assert_fp4_bitexact(g, oz, d, w.smooth_q)
+    rng = np.random.default_rng(16384)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 129, N - 1], rng.integers(0, N, 11)])).astype(np.int32)
+    ref = to_dtype_np(orc.attention_nvfp4(oz, w.causal, rows=rows), w.dtype)
+    got = out.float().cpu().reshape(B * H, N, d).numpy()[:, rows]
+    compare_out(got, ref, w.dtype, "nvfp4 full size")
