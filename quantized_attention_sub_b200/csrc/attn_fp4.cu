@@ -110,8 +110,11 @@ __global__ void __launch_bounds__(128)
 //               each with its block-scale atoms); owns the TMEM allocation
 //   warp 9      MMA issuer (one thread): copies scale atoms into TMEM
 //               (tcgen05.cp), S = Q K^T and O += P~ V with kind::mxf4nvf4
-// TMEM (512 columns): S double buffer [0,128) and [128,256), O [256,384),
-// block scales from 384: Q, K per stage, V per stage, P~ per buffer.
+// TMEM (256 columns, two CTAs per SM): S [0,64) holds one 64-key half of a
+// tile at a time (S = Q K_h^T, N = 64: the half's threads load it into
+// registers and free it for the other half), O [64,192), block scales from
+// 192: Q, K and V (two slots each, alternating by tile), P~ (per buffer).
+// The K scales of half h are the copied atom's columns 2h, 2h+1.
 // Per key tile j, the two threads of row i (one per key half):
 //   load their 64 S values, take the half's logit max, exchange it,
 //   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
@@ -127,7 +130,8 @@ __global__ void __launch_bounds__(128)
 constexpr int kStagesF = 3;
 constexpr int kSoftmaxWarpsF = 8, kProducerWarpF = 8, kMmaWarpF = 9;
 constexpr int kThreadsF = 320;
-constexpr uint32_t kColO = 256, kColSfq = 384, kColSfk = 392, kColSfv = 416, kColSfp = 440;
+constexpr uint32_t kTmemColsF = 256;
+constexpr uint32_t kColS = 0, kColO = 64, kColSfq = 192, kColSfk = 200, kColSfv = 216, kColSfp = 232;
 
 struct SmemF {
   static constexpr int kTile = 128 * 64;  // 128 rows x 64 bytes (d = 128 or 128 keys of e2m1)
@@ -161,7 +165,7 @@ struct AttnF4Args {
 enum : int { kErrProducerF = 0x311, kErrMmaF = 0x312, kErrSoftmaxF = 0x313, kErrDrainF = 0x314 };
 
 template <typename OutT, bool HAS_BIAS>
-__global__ void __launch_bounds__(kThreadsF, 1)
+__global__ void __launch_bounds__(kThreadsF, 2)
     attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnF4Args a) {
   using L = SmemF;
@@ -174,8 +178,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   uint64_t* k_empty = k_full + kStagesF;
   uint64_t* v_full = k_full + 2 * kStagesF;
   uint64_t* v_empty = k_full + 3 * kStagesF;
-  uint64_t* s_full = k_full + 4 * kStagesF;  // [2]
-  uint64_t* s_free = s_full + 2;             // [2]
+  uint64_t* s_full = k_full + 4 * kStagesF;  // [half 2]
+  uint64_t* s_free = s_full + 2;             // [half 2]
   uint64_t* p_full = s_full + 4;             // [2]
   uint64_t* o_done = s_full + 6;
   uint64_t* x_bar = s_full + 7;  // [2 parities]
@@ -200,7 +204,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], kSoftmaxWarpsF);
+      mbar_init(&s_free[b], kSoftmaxWarpsF / 2);  // the four warps of one half
       mbar_init(&p_full[b], kSoftmaxWarpsF);
       mbar_init(&x_bar[b], 256);
     }
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     fence_mbar_init();
   }
   if (warp == kProducerWarpF) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, kTmemColsF);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -259,7 +263,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   } else if (warp == kMmaWarpF) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_fp4(128, 128);
+      constexpr uint32_t idesc_s = idesc_fp4(128, 64);   // one 64-key half of S
+      constexpr uint32_t idesc_pv = idesc_fp4(128, 128);  // O += P~ V, N = d
       const uint32_t q_base = smem_u32(smem + L::off_q), k_base = smem_u32(smem + L::off_k);
       const uint32_t v_base = smem_u32(smem + L::off_v), p_base = smem_u32(smem + L::off_p);
       const uint32_t sfk_base = smem_u32(smem + L::off_sfk), sfv_base = smem_u32(smem + L::off_sfv);
@@ -269,49 +274,63 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int ka = 0; ka < 2; ++ka)
           tmem_cp_sf(tmem + kColSfq + 4 * ka, sf_atom_desc(smem_u32(smem + L::off_sfq) + 512 * ka));
       }
-      auto issue_s = [&](int j) {
+      // S(j) half h: keys [64h, 64h + 64) of tile j (rows 64h.. of the K tile;
+      // their scales are columns 2h, 2h+1 of the copied atoms)
+      auto issue_s = [&](int j, int h) {
         const int s = j % kStagesF;
-        const uint32_t kb = k_base + s * L::kTile, sfk = kColSfk + 8 * s;
-        for (int ka = 0; ka < 2; ++ka)
-          tmem_cp_sf(tmem + sfk + 4 * ka, sf_atom_desc(sfk_base + s * L::kSf + 512 * ka));
+        const uint32_t kb = k_base + s * L::kTile + h * 64 * 64, sfk = kColSfk + 8 * (j & 1);
+        if (h == 0)
+          for (int ka = 0; ka < 2; ++ka)
+            tmem_cp_sf(tmem + sfk + 4 * ka, sf_atom_desc(sfk_base + s * L::kSf + 512 * ka));
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
-          mma_fp4(tmem + 128 * (j & 1), kmajor_desc(q_base + kk * 32, 64), kmajor_desc(kb + kk * 32, 64), idesc,
-                  tmem + kColSfq + 4 * kk, tmem + sfk + 4 * kk, kk > 0);
-        tc_commit(&s_full[j & 1]);
+          mma_fp4(tmem + kColS, kmajor_desc(q_base + kk * 32, 64), kmajor_desc(kb + kk * 32, 64), idesc_s,
+                  tmem + kColSfq + 4 * kk, tmem + sfk + 4 * kk + 2 * h, kk > 0);
+        tc_commit(&s_full[h]);
       };
       auto issue_pv = [&](int j) {
         const int s = j % kStagesF;
-        const uint32_t pa = p_base + (j & 1) * L::kTile, vb = v_base + s * L::kTile, sfv = kColSfv + 8 * s;
+        const uint32_t pa = p_base + (j & 1) * L::kTile, vb = v_base + s * L::kTile, sfv = kColSfv + 8 * (j & 1);
         for (int ka = 0; ka < 2; ++ka)
           tmem_cp_sf(tmem + sfv + 4 * ka, sf_atom_desc(sfv_base + s * L::kSf + 512 * ka));
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
-          mma_fp4(tmem + kColO, kmajor_desc(pa + kk * 32, 64), kmajor_desc(vb + kk * 32, 64), idesc,
+          mma_fp4(tmem + kColO, kmajor_desc(pa + kk * 32, 64), kmajor_desc(vb + kk * 32, 64), idesc_pv,
                   tmem + kColSfp + 8 * (j & 1) + 4 * kk, tmem + sfv + 4 * kk, (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(o_done);
       };
+      // the S buffer passes S(j)_0 -> S(j)_1 -> S(j+1)_0 -> ..., each issued
+      // once the previous half has been loaded by its threads
       if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
-        tc_commit(&k_empty[0]);
+        issue_s(0, 0);
+        if ((ok = mbar_wait(&s_free[0], 0, abort_flag))) {
+          tc_fence_after();
+          issue_s(0, 1);
+          tc_commit(&k_empty[0]);
+        }
       }
       for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T) {
-          // S(j+1) into the buffer S(j-1) used, once the softmax has read it
-          const int s1 = (j + 1) % kStagesF;
+        const bool next = j + 1 < T;
+        const int s1 = (j + 1) % kStagesF;
+        if (next) {
           if (!(ok = mbar_wait(&k_full[s1], ((j + 1) / kStagesF) & 1, abort_flag))) break;
-          if (j >= 1 && !(ok = mbar_wait(&s_free[(j + 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&s_free[1], j & 1, abort_flag))) break;  // S(j)_1 loaded
           tc_fence_after();
-          issue_s(j + 1);
-          tc_commit(&k_empty[s1]);
+          issue_s(j + 1, 0);
         }
         if (!(ok = mbar_wait(&v_full[j % kStagesF], (j / kStagesF) & 1, abort_flag))) break;
         if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         issue_pv(j);
         tc_commit(&v_empty[j % kStagesF]);
+        if (next) {
+          if (!(ok = mbar_wait(&s_free[0], (j + 1) & 1, abort_flag))) break;  // S(j+1)_0 loaded
+          tc_fence_after();
+          issue_s(j + 1, 1);
+          tc_commit(&k_empty[s1]);
+        }
       }
       if (!ok) fail(abort_flag, a.err, kErrMmaF);
       // Every MMA issued so far must complete before the CTA frees TMEM.
@@ -342,19 +361,19 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         lim = min(lim, a.N - kbase);
         if (a.causal) lim = min(lim, row - kbase + 1);
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[h], j & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[64];
-      const uint32_t t_s = tmem + lane_off + 128 * (j & 1) + h * 64;
+      const uint32_t t_s = tmem + lane_off + kColS;
       tmem_ld32(t_s, sr);
       tmem_ld32(t_s + 32, sr + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[j & 1]);
+      if (lane == 0) mbar_arrive(&s_free[h]);
 
       // t = x kf (or fma(x, kf, bias log2(e)/sqrt(d))), the INT8 mode's steps
       if (lim < 64) {
@@ -515,7 +534,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   tc_fence_after();
   if (warp == kProducerWarpF) {
     __syncwarp();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemColsF);
   }
 }
 
