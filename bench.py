@@ -35,7 +35,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from quantized_attention_sub_b200 import api, inputs  # noqa: E402
+from quantized_attention_sub_b200 import api, inputs, replicas  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio 4.5 / 2.25 PFLOP/s (INT8 dense equals FP8 dense)
@@ -59,30 +59,15 @@ def load_peaks():
 
 
 def dist_init():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return ws, rank, local
+    return replicas.init("nccl")
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    replicas.barrier(ws)
 
 
 def allreduce_max(x, ws):
-    if ws == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return replicas.max_over_ranks(x, ws, "cuda")
 
 
 class ClockSampler:
@@ -215,7 +200,7 @@ def main():
     B, H, N, d = w.shape()
     dcode = api.DTYPE_CODE[inputs.DTYPES[w.dtype]]
     # each rank draws its own slice batch (seed offset by rank)
-    wr = inputs.variant(w, seed=w.seed + 7919 * rank)
+    wr = inputs.variant(w, seed=replicas.rank_seed(w.seed, rank))
     q, k, v = [t.to(dev) for t in inputs.generate(wr, device="cuda")]
     out = torch.empty_like(q)
     wsbuf = api.alloc_workspace(B, H, N, d, w.mode, dev)
@@ -261,7 +246,7 @@ def main():
 
     ops_visible = inputs.executed_ops(w) * ws
     ops_square = inputs.attention_ops(w) * ws
-    value = ops_visible / (ms * 1e-3) / 1e12
+    value = replicas.job_throughput(inputs.executed_ops(w), ms, ws) / 1e12
 
     # roofline of the dominant kernel (attention), live CUDA-event time
     peaks, peak_src = load_peaks()
@@ -321,7 +306,7 @@ def main():
             "quant_roofline": quant_line,
             "e2e": {"value": ops_visible / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes},
-            # per step: the stats, fold and codes quantization kernels and attn_i8f8_kernel
+            # per step: the stats, fold and codes quantization kernels and the attention kernel
             "gpu_launches": 4 * args.steps,
             "clocks": clk}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
