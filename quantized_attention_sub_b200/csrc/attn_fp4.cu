@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(kThreadsF, 2)
           const int c = 16 * cc + 4 * e;
           const float2 ga2 = make_float2(sat_fma(u2f(sr[c]), gm, cs), sat_fma(u2f(sr[c + 1]), gm, cs));
           const float2 gb2 = make_float2(sat_fma(u2f(sr[c + 2]), gm, cs), sat_fma(u2f(sr[c + 3]), gm, cs));
-          const float2 pa = exp2g2(ga2), pb = exp2g2(gb2);
+          const float2 pa = exp2g2<false>(ga2), pb = exp2g2<false>(gb2);
           sa = __fadd2_rn(sa, pa);
           sb = __fadd2_rn(sb, pb);
           p[4 * e] = pa.x;

@@ -30,12 +30,26 @@ SAGE_DEV float fmax3(float a, float b, float c) {
 
 // exp2 of the method, the same definition the CPU reference computation uses.
 // The argument is carried as g = (d + 127) / 256 saturated to [0, 1]; then
-// k = floor(256 g) (the round-down fma with 1.5*2^23 - 127 gives
-// 1.5*2^23 - 127 + k exactly), f = 256 g - k, 2^f by a degree-3 polynomial
-// with constant term 1 (Remez fit of the relative error, max 8.6e-5), and
-// k - 127 added to the exponent field.  Exact at integer d; d <= -127 gives +0.
+// k = floor(256 g) (the round-down fma with 1.5*2^23 gives 1.5*2^23 + k
+// exactly, so k sits in the low byte of its bits), f = 256 g - k, 2^f by a
+// degree-3 polynomial with constant term 1 (Remez fit of the relative error,
+// max 8.6e-5; its values lie in [1, 2), so its exponent field is 127), and
+// the exponent field replaced by k: 2^f * 2^(k - 127).  Exact at integer d;
+// d <= -127 gives +0.  Every caller keeps d < 129 (k <= 255).
+// Two equivalent ways to set that exponent are kept, since they schedule
+// differently: a bit-field insert of k (y = 1.5*2^23 + k), or adding
+// (k - 127) << 23 to the bits of 2^f (y = 1.5*2^23 - 127 + k); the kernels
+// pick per instantiation whichever measured faster.
 constexpr float kE1 = 0x1.63e658p-1f, kE2 = 0x1.d2378ap-3f, kE3 = 0x1.3baaa6p-4f;
-constexpr float kMg = 12582912.0f - 127.0f;
+constexpr float kMg = 12582912.0f;
+constexpr float kMgAdd = 12582912.0f - 127.0f;
+
+// r with its exponent field (bits 23..30) replaced by the low byte of y's bits.
+SAGE_DEV float set_exponent(float r, float y) {
+  uint32_t d;
+  asm("bfi.b32 %0, %1, %2, 23, 8;" : "=r"(d) : "r"(__float_as_uint(y)), "r"(__float_as_uint(r)));
+  return __uint_as_float(d);
+}
 
 SAGE_DEV float sat_fma(float a, float b, float c) {
   float d;
@@ -49,20 +63,24 @@ SAGE_DEV float exp2g(float g) {
   float r = __fmaf_rn(kE3, f, kE2);
   r = __fmaf_rn(r, f, kE1);
   r = __fmaf_rn(r, f, 1.0f);
-  return __uint_as_float(__float_as_uint(r) + (__float_as_uint(y) << 23));
+  return set_exponent(r, y);
 }
 
 // exp2 of a plain argument d (used for the rescale factor alpha).
 SAGE_DEV float exp2m(float d) { return exp2g(__saturatef(__fmul_rn(__fadd_rn(d, 127.0f), 0x1p-8f))); }
 
-// The same as exp2g on a pair, with the packed f32x2 ALU operations.
+// The same as exp2g on a pair, with the packed f32x2 ALU operations; BFI
+// selects the exponent insertion (the results are identical).
+template <bool BFI = true>
 SAGE_DEV float2 exp2g2(float2 g) {
-  const float2 y = __ffma2_rd(g, make_float2(256.0f, 256.0f), make_float2(kMg, kMg));
-  const float2 k = __fadd2_rn(y, make_float2(-kMg, -kMg));
+  constexpr float M = BFI ? kMg : kMgAdd;
+  const float2 y = __ffma2_rd(g, make_float2(256.0f, 256.0f), make_float2(M, M));
+  const float2 k = __fadd2_rn(y, make_float2(-M, -M));
   const float2 f = __ffma2_rn(g, make_float2(256.0f, 256.0f), make_float2(-k.x, -k.y));
   float2 r = __ffma2_rn(make_float2(kE3, kE3), f, make_float2(kE2, kE2));
   r = __ffma2_rn(r, f, make_float2(kE1, kE1));
   r = __ffma2_rn(r, f, make_float2(1.0f, 1.0f));
+  if (BFI) return make_float2(set_exponent(r.x, y.x), set_exponent(r.y, y.y));
   return make_float2(__uint_as_float(__float_as_uint(r.x) + (__float_as_uint(y.x) << 23)),
                      __uint_as_float(__float_as_uint(r.y) + (__float_as_uint(y.y) << 23)));
 }
