@@ -41,6 +41,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_OVER_BF16 = 2.0   # nominal dense ratio 4.5 / 2.25 PFLOP/s (INT8 dense equals FP8 dense)
 FP4_OVER_BF16 = 4.0   # nominal dense ratio 9 / 2.25 PFLOP/s
 
+# DRAM bytes (read + write) of one attention launch at the workload's full
+# size, from one ncu capture of the kernel as it stands on a smaller case
+# (inputs still above L2), scaled by the token count (attention traffic is
+# the codes read once plus the output, linear in N).  null for other sizes.
+TRAFFIC_BYTES = {"llm_prefill": 124.1e6, "video_dit": 196.0e6, "nvfp4": 64.4e6}
+
 # per mode: tensor peak ratio to bf16, attention kernel, arithmetic description
 MODE_INFO = {
     0: (FP8_OVER_BF16, "attn_i8f8_kernel", "int8 QK / e4m3 PV, fp32 softmax and accumulation"),
@@ -178,6 +184,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llm_prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--N", type=int, default=0,
+                    help="override the workload's sequence length (small cases for profiling; "
+                         "the headline runs use the workload's own N)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -186,6 +195,8 @@ def main():
     if w is None and args.workload.startswith("sweep_"):
         _, n, d, c = args.workload.split("_")
         w = inputs.sweep(int(n[1:]), int(d[1:]), c == "causal")
+    if args.N > 0:
+        w = inputs.variant(w, N=args.N)
     ws, rank, local = dist_init() if args.impl == "ours" or int(os.environ.get("WORLD_SIZE", "1")) > 1 else (1, 0, 0)
 
     if args.impl == "reference":
@@ -257,7 +268,8 @@ def main():
                 "unit": "TFLOP/s", "frac": achieved / peak_fp8,
                 "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense %s : BF16 ratio)" % (
                     peak_src, ratio, "FP4" if w.mode == 2 else "FP8/INT8"),
-                "traffic": None, "attn_ms": attn_avg}
+                "traffic": TRAFFIC_BYTES.get(w.name) if args.N == 0 else None,
+                "traffic_unit": "bytes per launch", "attn_ms": attn_avg}
     # the quantization pass (HBM-bound): 16-bit Q, K, V read once, int8/e4m3
     # codes written, statistics and scales (small) not counted
     Np = (N + 127) // 128 * 128

@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kThreadsF, 2)
       // the previous tile's rescale) and the four scales into TMEM
       uint8_t* prow = prow0 + (j & 1) * L::kTile;
       float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-      uint32_t cw[8];
+      uint32_t cw[4];
       uint32_t sfw = 0;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -455,12 +455,12 @@ __global__ void __launch_bounds__(kThreadsF, 2)
         const float rr = sd > 0.f ? __fdiv_rn(1.0f, __fmul_rn(gp, sd)) : 0.f;
 #pragma unroll
         for (int e = 0; e < 16; ++e) p[e] = __fmul_rn(p[e], rr);
-        cw[2 * cc] = e2m1x8(p);
-        cw[2 * cc + 1] = e2m1x8(p + 8);
+        cw[2 * (cc & 1)] = e2m1x8(p);
+        cw[2 * (cc & 1) + 1] = e2m1x8(p + 8);
         sfw |= bs << (8 * cc);
+        if (cc & 1)  // a 16-byte chunk (32 keys) is complete
+          *reinterpret_cast<uint4*>(prow + (((2 * h + (cc >> 1)) ^ swz) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       }
-      *reinterpret_cast<uint4*>(prow + (((2 * h) ^ swz) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      *reinterpret_cast<uint4*>(prow + (((2 * h + 1) ^ swz) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
       tmem_st1(tmem + lane_off + kColSfp + 8 * (j & 1) + 4 * h + w4, sfw);
       fence_proxy_async_smem();
       if (j > 0) {
