@@ -118,7 +118,7 @@ def f16_round(x: float) -> float:
 
 
 def exp2(d: float) -> float:
-    """The exp2 both sides use (range reduction + degree-4 polynomial)."""
+    """The softmax's exp2: the library exp2 in double, rounded to fp32."""
     return lib().orc_exp2(float(d))
 
 

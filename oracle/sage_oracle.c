@@ -153,46 +153,14 @@ ORC_EXPORT double orc_f16_round(double x)
   return x < 0 ? -r : r;
 }
 
-/* exp2 as both sides compute it.  The pages fix no accuracy for the softmax
- * exponential; this reading fixes one, so that the FP8 decision P~ =
- * e4m3(2^d) is the same bit for bit on the CPU and on the GPU.
- *
- * The argument is carried as g = (d + 127) / 256, saturated to [0, 1] (NaN
- * gives 0): d <= -127 gives +0 and the largest d the softmax produces
- * (log2(448) < 9) stays inside.  Then k = floor(256 g) and f = 256 g - k (both
- * exact in fp32), 2^f by a degree-3 polynomial with its constant term fixed to
- * 1 (coefficients from a Remez exchange on the relative error; max relative
- * error 8.6e-5 in fp32 Horner form, far below the 2^-4 step of e4m3; exact at
- * integers, so a row max that does not move gives alpha = 1), and k - 127
- * added to the exponent field (k = 0 gives +0). */
-static const float EXP2_C1 = 0x1.63e658p-1f;
-static const float EXP2_C2 = 0x1.d2378ap-3f;
-static const float EXP2_C3 = 0x1.3baaa6p-4f;
-
-static float sat01(float g)
-{
-  if (!(g > 0.0f)) return 0.0f;   /* NaN included */
-  return g < 1.0f ? g : 1.0f;
-}
-
-/* 2^(256 g - 127) for g already saturated to [0, 1]. */
-static float exp2_g(float g)
-{
-  float k = floorf(g * 256.0f);
-  float f = g * 256.0f - k;
-  float r = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.0f);
-  uint32_t rb;
-  memcpy(&rb, &r, 4);
-  rb += ((uint32_t)(int32_t)k - 127u) << 23;
-  float out;
-  memcpy(&out, &rb, 4);
-  return out;
-}
-
-/* exp2 of a plain argument: g = fl(d + 127) / 256. */
+/* exp2 of the softmax: the library exp2 in double, rounded once to fp32.
+ * The pages fix no accuracy for the exponential; the GPU evaluates it on its
+ * special-function unit (ex2.approx), whose result may differ from this one
+ * in the last bits, so a P~ code can differ in rare cases and the attention
+ * output is compared within a tolerance.  -inf gives +0. */
 ORC_EXPORT float orc_exp2(float d)
 {
-  return exp2_g(sat01((d + 127.0f) * 0x1p-8f));
+  return (float)exp2((double)d);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -358,10 +326,9 @@ enum { ORC_MODE_FP32ACC = 0, ORC_MODE_F16ACC = 1 };
  *   kf    = (sq_i * sk_g(j)) * (log2(e) / sqrt(d))        one factor per 64-key granule
  *   t_j   = float(S_ij) * kf, or fma(float(S_ij), kf, bias_j * (log2(e)/sqrt(d)))
  *   m_new = max(m, max_j t_j);  alpha = exp2(m - m_new);  m' = m_new - log2(Pr)
- *   p'_j  = exp2(t_j - m') = p_j * Pr with p_j the softmax numerator, where the
- *           argument is formed in one rounding together with the +127 offset of
- *           the exp2 below: g_j = fma(float(S_ij), kf / 256, (127 - m') / 256)
- *           (or fma(t_j, 1/256, (127 - m') / 256) with a bias);
+ *   p'_j  = exp2(d_j) = p_j * Pr with p_j the softmax numerator, where
+ *           d_j = fma(float(S_ij), kf, -m') in one rounding (t_j - m' with a
+ *           bias);
  *   l     = alpha * l + sum_j p'_j        (in units of Pr)
  *   P~_j  = e4m3(p'_j)
  *   FP32 accumulator: acc_c = alpha * acc_c + fl32(exact sum_j P~_j v^_jc)
@@ -399,15 +366,14 @@ static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* v
     const float m_new = m > mt ? m : mt;
     const float alpha = orc_exp2(m - m_new);   /* first tile: exp2(-inf) = 0 */
     const float mp = m_new - log2Pr;
-    /* d_j = t_j - m' + 127 in one rounding, carried as g = d / 256 */
-    const float cs = (127.0f - mp) * 0x1p-8f;
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
       float p = 0.0f;
       if (j0 + j <= jmax) {
+        /* d = t - m' (without bias in one rounding: fma(x, kf, -m')) */
         const float kf = (sq * sk[(j0 + j) / 64]) * c_log2;
-        const float g = bias ? fmaf(tvals[j], 0x1p-8f, cs) : fmaf(xvals[j], kf * 0x1p-8f, cs);
-        p = exp2_g(sat01(g));
+        const float dd = bias ? tvals[j] - mp : fmaf(xvals[j], kf, -mp);
+        p = orc_exp2(dd);
       }
       ps = ps + p;
       pcode[j] = orc_e4m3_encode((double)p);
@@ -589,14 +555,12 @@ static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq
     }
     const float m_new = m > mt ? m : mt;
     const float alpha = orc_exp2(m - m_new);
-    /* d_j = t_j - m_new + 127 in one rounding, carried as g = d / 256 */
-    const float cs = (127.0f - m_new) * 0x1p-8f;
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
       float p = 0.0f;
       if (j0 + j <= jmax) {
-        const float g = bias ? fmaf(tvals[j], 0x1p-8f, cs) : fmaf(xvals[j], kf * 0x1p-8f, cs);
-        p = exp2_g(sat01(g));
+        const float dd = bias ? tvals[j] - m_new : fmaf(xvals[j], kf, -m_new);
+        p = orc_exp2(dd);
       }
       pvals[j] = p;
       ps = ps + p;

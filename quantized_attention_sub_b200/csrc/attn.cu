@@ -18,13 +18,14 @@
 //   load their 64 S values from TMEM and free the S buffer,
 //   take the half's logit max and exchange it through shared memory,
 //   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
-//   p' = exp2(d) with d = t - m_new + log2(Pr), P~ = e4m3(p'),
+//   p' = 2^d with d = t - m_new + log2(Pr), P~ = e4m3(p'),
 //   wait for the previous P~V, multiply their half of the O row by alpha
 //   (skipped when alpha == 1 on the whole warp), write their 64 P~ bytes into
 //   the 128B-swizzled K-major shared tile the MMA reads, l_h = alpha l_h + sum p'.
 // At the end l = l_0 + l_1 and O = acc * scale_v / l is cast and stored.
-// exp2 is the method's own (range reduction + degree-3 polynomial), so the P~
-// codes equal those of the CPU reference computation bit for bit.
+// exp2 runs on the special-function unit (ex2.approx); the CPU reference
+// computation uses the library exp2, so a P~ code may differ in rare cases and
+// the output is compared within a tolerance.
 // Every wait is bounded (sage_ptx.cuh); a timeout records an error code in
 // the workspace, makes the other roles stop, and the CTA frees its TMEM.
 #include <cuda_bf16.h>
@@ -347,16 +348,15 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
 
-        // Logits and P~ follow the method's fp32 steps exactly (the CPU
-        // reference computation takes the same ones):
+        // Logits and P~ take the fp32 steps of the CPU reference computation:
         //   kf = (sq * sk) * log2(e)/sqrt(d) for this half's 64-key granule,
         //   t  = float(S) * kf  (or fma(float(S), kf, bias * log2(e)/sqrt(d))),
-        //   m' = max - log2(Pr),  g = sat(fma(float(S), kf/256, (127 - m')/256))
-        //   (or sat(fma(t, 1/256, (127 - m')/256))),  p' = exp2g(g) = p * Pr,
-        //   P~ = e4m3(p').
-        // Masked keys become -inf: out of the max, and g saturates to 0 (also
-        // from NaN, for a zero scale), where exp2g gives +0.
-        const float kf = __fmul_rn(__fmul_rn(sq, h ? ks.y : ks.x), a.c_log2);
+        //   m' = max - log2(Pr),  d = fma(float(S), kf, -m')  (or t - m'),
+        //   p' = 2^d = p * Pr on the special-function unit, P~ = e4m3(p').
+        // Masked keys become -inf: out of the max, and 2^-inf = +0.  (A zero
+        // scale -- an all-zero granule -- is raised to the smallest normal
+        // float so that masked keys stay at -inf instead of NaN.)
+        const float kf = fmaxf(__fmul_rn(__fmul_rn(sq, h ? ks.y : ks.x), a.c_log2), 1.17549435e-38f);
 #pragma unroll
         for (int c = 0; c < 64; ++c) sr[c] = f2u(__int2float_rn((int)sr[c]));
         if (lim < 64) {
@@ -406,10 +406,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         }
         mt = fmaxf(mt, xs[(h ^ 1) * 128 + r]);
         const float m_new = fmaxf(m, mt);
-        const float alpha = exp2m(__fadd_rn(m, -m_new));  // +0 on the first tile (m = -inf), 1 if the max stays
-        const float mp = m_new - a.log2Pr;
-        const float cs = __fmul_rn(__fadd_rn(127.0f, -mp), 0x1p-8f);
-        const float gm = HAS_BIAS ? 0x1p-8f : __fmul_rn(kf, 0x1p-8f);
+        const float alpha = ex2(__fadd_rn(m, -m_new));  // +0 on the first tile (m = -inf), 1 if the max stays
+        const float mp = __fadd_rn(m_new, -a.log2Pr);
+        const float2 nmp = make_float2(-mp, -mp), kf2 = make_float2(kf, kf);
 
         // p' = p * Pr for the 64 keys, P~ = e4m3(p') packed 4 per word and
         // stored 16 keys at a time into this tile's P buffer (the buffer was
@@ -423,9 +422,11 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 16 * cc + 4 * e;
-            const float2 ga2 = make_float2(sat_fma(u2f(sr[c]), gm, cs), sat_fma(u2f(sr[c + 1]), gm, cs));
-            const float2 gb2 = make_float2(sat_fma(u2f(sr[c + 2]), gm, cs), sat_fma(u2f(sr[c + 3]), gm, cs));
-            const float2 pa = exp2g2<!F16ACC>(ga2), pb = exp2g2<!F16ACC>(gb2);
+            // d = t - m' (one rounding: fma(x, kf, -m') without bias)
+            const float2 xa = make_float2(u2f(sr[c]), u2f(sr[c + 1])), xb = make_float2(u2f(sr[c + 2]), u2f(sr[c + 3]));
+            const float2 da = HAS_BIAS ? __fadd2_rn(xa, nmp) : __ffma2_rn(xa, kf2, nmp);
+            const float2 db = HAS_BIAS ? __fadd2_rn(xb, nmp) : __ffma2_rn(xb, kf2, nmp);
+            const float2 pa = make_float2(ex2(da.x), ex2(da.y)), pb = make_float2(ex2(db.x), ex2(db.y));
             sa = __fadd2_rn(sa, pa);
             sb = __fadd2_rn(sb, pb);
             pw[e] = e4m3x4(pa, pb);

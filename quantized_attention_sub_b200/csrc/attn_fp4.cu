@@ -118,8 +118,8 @@ __global__ void __launch_bounds__(128)
 // Per key tile j, the two threads of row i (one per key half):
 //   load their 64 S values, take the half's logit max, exchange it,
 //   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
-//   p = exp2(t - m_new) (the method's exp2, the same argument steps as the
-//   INT8 mode), l_h = alpha l_h + sum p,
+//   p = exp2(t - m_new) on the special-function unit (the argument in the
+//   INT8 mode's steps), l_h = alpha l_h + sum p,
 //   per 16 keys: bs = ue4m3(max p / (6 g_p)), r = 1 / (g_p dec(bs)),
 //   P~ = e2m1(p r): 32 bytes of codes into the 64-byte swizzled P~ row and
 //   one 32-bit word of four scales into TMEM (tcgen05.st),
@@ -348,7 +348,9 @@ __global__ void __launch_bounds__(kThreadsF, 2)
     uint8_t* prow0 = smem + L::off_p + r * 64;  // buffer 0; buffer 1 is kTile further
     const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
     const float4 gsc = *reinterpret_cast<const float4*>(a.gscale + (size_t)bh * 4);  // g_q, g_k, g_v, 0
-    const float kf = __fmul_rn(__fmul_rn(gsc.x, gsc.y), a.c_log2);
+    // (a zero global scale -- an all-zero Q or K slice -- is raised to the
+    // smallest normal float so that masked keys stay at -inf instead of NaN)
+    const float kf = fmaxf(__fmul_rn(__fmul_rn(gsc.x, gsc.y), a.c_log2), 1.17549435e-38f);
     const float gp = __fdiv_rn(1.0f, 2688.0f);  // P~ global scale 1 / (6 * 448)
     const float six_gp = __fmul_rn(6.0f, gp);
     const int swz = (r >> 1) & 3;  // 64-byte swizzle of this row's 16-byte chunks
@@ -420,9 +422,8 @@ __global__ void __launch_bounds__(kThreadsF, 2)
       }
       mt = fmaxf(mt, xs[(h ^ 1) * 128 + r]);
       const float m_new = fmaxf(m, mt);
-      const float alpha = exp2m(__fadd_rn(m, -m_new));
-      const float cs = __fmul_rn(__fadd_rn(127.0f, -m_new), 0x1p-8f);
-      const float gm = HAS_BIAS ? 0x1p-8f : __fmul_rn(kf, 0x1p-8f);
+      const float alpha = ex2(__fadd_rn(m, -m_new));
+      const float2 nm2 = make_float2(-m_new, -m_new), kf2 = make_float2(kf, kf);
 
       // p for the 64 keys, then per 16 keys the FP4 block: P~ codes into this
       // tile's P buffer (last read by the P~V two tiles back, complete before
@@ -437,9 +438,11 @@ __global__ void __launch_bounds__(kThreadsF, 2)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c = 16 * cc + 4 * e;
-          const float2 ga2 = make_float2(sat_fma(u2f(sr[c]), gm, cs), sat_fma(u2f(sr[c + 1]), gm, cs));
-          const float2 gb2 = make_float2(sat_fma(u2f(sr[c + 2]), gm, cs), sat_fma(u2f(sr[c + 3]), gm, cs));
-          const float2 pa = exp2g2<false>(ga2), pb = exp2g2<false>(gb2);
+          // d = t - m_new (without bias in one rounding: fma(x, kf, -m_new))
+          const float2 xa = make_float2(u2f(sr[c]), u2f(sr[c + 1])), xb = make_float2(u2f(sr[c + 2]), u2f(sr[c + 3]));
+          const float2 da = HAS_BIAS ? __fadd2_rn(xa, nm2) : __ffma2_rn(xa, kf2, nm2);
+          const float2 db = HAS_BIAS ? __fadd2_rn(xb, nm2) : __ffma2_rn(xb, kf2, nm2);
+          const float2 pa = make_float2(ex2(da.x), ex2(da.y)), pb = make_float2(ex2(db.x), ex2(db.y));
           sa = __fadd2_rn(sa, pa);
           sb = __fadd2_rn(sb, pb);
           p[4 * e] = pa.x;
