@@ -237,13 +237,16 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
     const bool need_q = PASS == kCodesPass || a.smooth_q || FP4;
     for (int it = 0;; ++it) {
       const int b = it & 1;
-      const int item = blockIdx.x + it * gridDim.x;
+      // the codes pass walks the items backwards: the slices the statistics
+      // pass read last are the likeliest to be still in L2
+      const int idx = blockIdx.x + it * gridDim.x;
+      const int item = PASS == kCodesPass ? a.n_items - 1 - idx : idx;
       if (it >= 2 && !mbar_wait(&empty[b], ((it >> 1) - 1) & 1, &abort_s)) {
         atomicCAS(a.err, 0, kErrTileWait);
         abort_s = 1;
         return;
       }
-      if (item >= a.n_items) {
+      if (idx >= a.n_items) {
         info[b] = make_int4(-1, 0, 0, 0);
         mbar_arrive(&full[b]);
         return;
