@@ -334,6 +334,13 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           lim = min(lim, a.N - kbase);
           if (a.causal) lim = min(lim, row - kbase + 1);
         }
+        // the tile's 64 bias values, loaded before the wait for S hides their latency
+        float4 bv[HAS_BIAS ? 16 : 1];
+        if (HAS_BIAS) {
+          const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
+#pragma unroll
+          for (int c4 = 0; c4 < 16; ++c4) bv[c4] = __ldg(b4 + c4);
+        }
         // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
         if (!__all_sync(0xffffffffu, mbar_wait(&s_full[q], j & 1, abort_flag))) {
           ok = false;
@@ -375,17 +382,15 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           // a half with no visible key gives -inf, or NaN for a zero scale
           mt = __fmul_rn(fmaxf(ga, gb), kf);
         } else {
-          const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
           float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
-            const float4 bv = __ldg(b4 + c4);
             const int c = 4 * c4;
             const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
-                                         __fmul2_rn(make_float2(bv.x, bv.y), cl2));
+                                         __fmul2_rn(make_float2(bv[c4].x, bv[c4].y), cl2));
             const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf),
-                                         __fmul2_rn(make_float2(bv.z, bv.w), cl2));
+                                         __fmul2_rn(make_float2(bv[c4].z, bv[c4].w), cl2));
             sr[c] = f2u(ta.x);
             sr[c + 1] = f2u(ta.y);
             sr[c + 2] = f2u(tb.x);
