@@ -431,7 +431,13 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
             const float2 xa = make_float2(u2f(sr[c]), u2f(sr[c + 1])), xb = make_float2(u2f(sr[c + 2]), u2f(sr[c + 3]));
             const float2 da = HAS_BIAS ? __fadd2_rn(xa, nmp) : __ffma2_rn(xa, kf2, nmp);
             const float2 db = HAS_BIAS ? __fadd2_rn(xb, nmp) : __ffma2_rn(xb, kf2, nmp);
-            const float2 pa = make_float2(ex2(da.x), ex2(da.y)), pb = make_float2(ex2(db.x), ex2(db.y));
+            // FP16 mode: 2 of every 8 pairs take the polynomial, the rest the
+            // special-function unit (measured: the best split with two
+            // softmax warps per SM sub-partition; the FP32 mode, with four,
+            // is bound by instruction issue and keeps all on the unit)
+            constexpr int kPolyPairs = F16ACC ? 2 : 0;
+            const float2 pa = (2 * e) < kPolyPairs ? ex2_poly2(da) : make_float2(ex2(da.x), ex2(da.y));
+            const float2 pb = (2 * e + 1) < kPolyPairs ? ex2_poly2(db) : make_float2(ex2(db.x), ex2(db.y));
             sa = __fadd2_rn(sa, pa);
             sb = __fadd2_rn(sb, pb);
             pw[e] = e4m3x4(pa, pb);

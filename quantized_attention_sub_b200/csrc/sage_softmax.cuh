@@ -64,6 +64,27 @@ SAGE_DEV float2 h2f2(uint32_t u) {
 SAGE_DEV float u2f(uint32_t u) { return __uint_as_float(u); }
 SAGE_DEV uint32_t f2u(float f) { return __float_as_uint(f); }
 
+// 2^d for two arguments on the FMA and ALU pipes, to share the softmax's
+// exponentials with the special-function unit.  d is clamped to -127 (masked
+// keys, d = -inf, give +0), split as d = n + f with n = rint(d) (adding
+// 1.5 * 2^23 leaves n in the low bits) and f in [-1/2, 1/2]; 2^f is a degree-5
+// polynomial with p(0) = 1 fitted by Remez exchange for least relative error
+// on [-1/2, 1/2] (at most 4.9e-7 evaluated in fp32, comparable to ex2.approx),
+// and n is added to the exponent field.  For d >= -127 the result is 2^d to
+// that accuracy (a denormal or +0 below 2^-126); d is at most 2^9 here.
+SAGE_DEV float2 ex2_poly2(float2 d) {
+  const float2 lo = make_float2(fmaxf(d.x, -127.0f), fmaxf(d.y, -127.0f));
+  const float2 t = __fadd2_rn(lo, make_float2(kMagicF, kMagicF));
+  const float2 f = __fadd2_rn(lo, __fadd2_rn(make_float2(kMagicF, kMagicF), make_float2(-t.x, -t.y)));
+  float2 q = __ffma2_rn(f, make_float2(0x1.23a604p-10f, 0x1.23a604p-10f), make_float2(0x1.3cbea8p-7f, 0x1.3cbea8p-7f));
+  q = __ffma2_rn(q, f, make_float2(0x1.c74322p-5f, 0x1.c74322p-5f));
+  q = __ffma2_rn(q, f, make_float2(0x1.ebfa4ep-3f, 0x1.ebfa4ep-3f));
+  q = __ffma2_rn(q, f, make_float2(0x1.62e39ep-1f, 0x1.62e39ep-1f));
+  const float2 p = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+  // the bits of t are kMagicI + n: shifted left by 23 only n << 23 remains
+  return make_float2(u2f(f2u(p.x) + (f2u(t.x) << 23)), u2f(f2u(p.y) + (f2u(t.y) << 23)));
+}
+
 template <typename OutT>
 SAGE_DEV uint32_t pack2(float a, float b);
 template <>
