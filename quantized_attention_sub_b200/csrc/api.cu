@@ -207,8 +207,11 @@ sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v
                      "static quantize launch");
 }
 
-sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
-                                int causal, int smooth_q, int mode, sage_stream_t stream) {
+// The attention launch behind sage_attn_quantized and sage_attn_fwd.  After
+// sage_quantize_qkv on the same stream (sage_attn_fwd) the workspace error
+// word is already clear; called on its own it clears it first.
+static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
+                                  int causal, int smooth_q, int mode, sage_stream_t stream, bool after_quantize) {
   sage_status st = check_shape(B, H, N, d, mode);
   if (st != SAGE_OK) return st;
   if (!out) return set_err(SAGE_ERR_INVALID_ARG, "null output pointer%s");
@@ -219,16 +222,24 @@ sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int 
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
   if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
-  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+  if (!after_quantize &&
+      (st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
   if (mode == SAGE_MODE_NVFP4)
-    return cuda_status(sage::launch_attn_fp4(resolve(const_cast<void*>(ws), L), out, pb, (cudaStream_t)stream),
-                       "attention launch");
+    return cuda_status(
+        sage::launch_attn_fp4(resolve(const_cast<void*>(ws), L), out, pb, (cudaStream_t)stream),
+        "attention launch");
   // Pr: full e4m3 range with the FP32 accumulator, 224 with the FP16 one
   // (SageAttention2++ summary, Sec. 3.1)
   const float Pr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 224.0f : 448.0f;
-  return cuda_status(sage::launch_attn_i8f8(resolve(const_cast<void*>(ws), L), out, pb, Pr, (cudaStream_t)stream),
-                     "attention launch");
+  return cuda_status(
+      sage::launch_attn_i8f8(resolve(const_cast<void*>(ws), L), out, pb, Pr, (cudaStream_t)stream),
+      "attention launch");
+}
+
+sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
+                                int causal, int smooth_q, int mode, sage_stream_t stream) {
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream, false);
 }
 
 sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
@@ -236,7 +247,7 @@ sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out
                           sage_stream_t stream) {
   sage_status st = sage_quantize_qkv(q, k, v, dtype, B, H, N, d, smooth_q, mode, ws, ws_bytes, stream);
   if (st != SAGE_OK) return st;
-  return sage_attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream);
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream, true);
 }
 
 sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,

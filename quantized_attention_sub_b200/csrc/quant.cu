@@ -227,6 +227,10 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
     fence_mbar_init();
   }
   __syncthreads();
+  // the codes pass may start while the fold kernel runs (programmatic
+  // launch): nothing it wrote is read before this point
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == kComputeWarps) {
     // ------------------------------------------------------------- loader
@@ -781,6 +785,9 @@ __global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
     fence_mbar_init();
   }
   __syncthreads();
+  // launched while the statistics pass may still run: wait for its partials
+  grid_dep_wait();
+  grid_dep_launch();
   Folder<D> f{piece, bar, &abort_s};
   const float* src = a.part + ((size_t)which * a.BH + bh) * nchunks * D;
   float acc;
@@ -819,6 +826,9 @@ __global__ void __launch_bounds__(D) quant_fold_fp4_kernel(const QuantArgs a) {
     fence_mbar_init();
   }
   __syncthreads();
+  // launched while the statistics pass may still run: wait for its partials
+  grid_dep_wait();
+  grid_dep_launch();
   Folder<D> f{piece, bar, &abort_s};
   auto src = [&](int pl) { return a.part + pl * plane + (size_t)bh * nchunks * D; };
   bool ok = true;
@@ -937,15 +947,18 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
     e = cudaMemsetAsync(w.v_scale, 0, (size_t)pb.BH * pb.Npad * 8, s);
     if (e != cudaSuccess) return e;
   }
+  // The statistics pass follows whatever the caller enqueued and launches
+  // normally; the fold and the codes pass follow this library's own kernels
+  // and launch programmatically (each waits for its predecessor's results).
   quant_pass_kernel<T, D, kStatsPass, FP4><<<g0, kThreadsQ, smem, s>>>(tq, tk, tv, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (FP4)
-    quant_fold_fp4_kernel<D><<<dim3(pb.BH, 3), D, 0, s>>>(a);
+    e = launch_kernel(quant_fold_fp4_kernel<D>, dim3(pb.BH, 3), dim3(D), 0, s, true, a);
   else
-    quant_fold_kernel<D><<<dim3(pb.BH, pb.smooth_q ? 3 : 2), D, 0, s>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  quant_pass_kernel<T, D, kCodesPass, FP4><<<g1, kThreadsQ, smem, s>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+    e = launch_kernel(quant_fold_kernel<D>, dim3(pb.BH, pb.smooth_q ? 3 : 2), dim3(D), 0, s, true, a);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(quant_pass_kernel<T, D, kCodesPass, FP4>, dim3(g1), dim3(kThreadsQ), smem, s, true, tq, tk,
+                       tv, a);
 }
 
 }  // namespace

@@ -29,6 +29,25 @@ struct Problem {
   int BH, N, Npad, d, dtype, smooth_q, mode, causal;
 };
 
+// Launch `kern` on `s`; with `pdl` it may start while the previous kernel on
+// the stream is still running (programmatic stream serialization): the kernel
+// must call grid_dep_wait before it reads what that kernel wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                                 Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Floats of scratch the quantization pass needs.  INT8/FP8 modes: statistics
 // partials [3][BH][Npad/64][d] (K sums, Q sums, |V| maxima) and V multipliers
 // [BH][d].  NVFP4: partials [7][BH][Npad/64][d] (the same three planes, then
@@ -45,7 +64,8 @@ cudaError_t launch_quant_static(const void* q, const void* k, const void* v, con
                                 cudaStream_t s);
 size_t static_scratch_floats();
 
-// Fused attention (FP32 PV accumulator).
+// Fused attention (FP32 or FP16 PV accumulator).  Launched normally: a
+// programmatic launch behind the codes pass measured slower on video_dit.
 cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s);
 
 // Fused NVFP4 attention (kind::mxf4nvf4 for S and P~V, FP32 accumulator); d = 128.

@@ -87,6 +87,14 @@ SAGE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return false;
 }
 
+// Programmatic dependent launch.  grid_dep_wait: block until the grids this
+// one depends on have completed and their memory is visible (returns at once
+// for a grid launched without the programmatic attribute).  grid_dep_launch:
+// let the next grid on the stream, if launched with the attribute, start its
+// CTAs (they run up to their own grid_dep_wait).
+SAGE_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SAGE_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 SAGE_DEV void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
