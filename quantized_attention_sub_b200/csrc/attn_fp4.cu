@@ -145,7 +145,8 @@ struct SmemF {
   static constexpr int off_p = off_sfv + kStagesF * kSf;  // [buffer 2]
   static constexpr int off_bar = off_p + 2 * kTile;
   static constexpr int off_x = off_bar + 256;  // [parity 2][half 2][row 128] floats
-  static constexpr int bytes = off_x + 2 * 2 * 128 * 4;
+  static constexpr int off_rtab = off_x + 2 * 2 * 128 * 4;  // [128] P~ block reciprocals
+  static constexpr int bytes = off_rtab + 128 * 4;
   static constexpr int alloc = bytes + 1024;
 };
 static_assert(SmemF::off_k % 1024 == 0 && SmemF::off_v % 1024 == 0 && SmemF::off_p % 1024 == 0, "tile alignment");
@@ -212,6 +213,13 @@ __global__ void __launch_bounds__(kThreadsF, 2)
     mbar_init(mma_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (threadIdx.x < 128) {
+    // P~ block reciprocal for every non-negative ue4m3 scale code b:
+    // RN(1 / RN(g_p * dec(b))), 0 for a zero scale (all 16 p of the block 0)
+    const float sd = e4m3_to_f32(threadIdx.x);
+    reinterpret_cast<float*>(smem + L::off_rtab)[threadIdx.x] =
+        sd > 0.f ? __fdiv_rn(1.0f, __fmul_rn(__fdiv_rn(1.0f, 2688.0f), sd)) : 0.f;
   }
   if (warp == kProducerWarpF) {
     tmem_alloc(tmem_slot, kTmemColsF);
@@ -353,6 +361,8 @@ __global__ void __launch_bounds__(kThreadsF, 2)
     const float kf = fmaxf(__fmul_rn(__fmul_rn(gsc.x, gsc.y), a.c_log2), 1.17549435e-38f);
     const float gp = __fdiv_rn(1.0f, 2688.0f);  // P~ global scale 1 / (6 * 448)
     const float six_gp = __fmul_rn(6.0f, gp);
+    const float inv_six_gp = __fdiv_rn(1.0f, six_gp);
+    const float* rtab = reinterpret_cast<const float*>(smem + L::off_rtab);
     const int swz = (r >> 1) & 3;  // 64-byte swizzle of this row's 16-byte chunks
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -453,11 +463,21 @@ __global__ void __launch_bounds__(kThreadsF, 2)
         float am = 0.f;
 #pragma unroll
         for (int e = 0; e < 16; e += 2) am = fmax3(am, p[e], p[e + 1]);
-        const uint32_t bs = e4m3x2(__fdiv_rn(am, six_gp), 0.f) & 0xFFu;
-        const float sd = e4m3_to_f32(bs);
-        const float rr = sd > 0.f ? __fdiv_rn(1.0f, __fmul_rn(gp, sd)) : 0.f;
+        // bs = ue4m3(am / (6 g_p)).  The quotient is formed as q0 = am * RN(1/c)
+        // with one FMA correction (Markstein's division by a correctly rounded
+        // reciprocal); over every float am in [0, 1] (p <= 1) it gives the same
+        // e4m3 code as the correctly rounded quotient (exhaustive check; the
+        // quotients differ only below the e4m3 range, for subnormal am).
+        const float q0 = __fmul_rn(am, inv_six_gp);
+        const float qd = __fmaf_rn(__fmaf_rn(-six_gp, q0, am), inv_six_gp, q0);
+        const uint32_t bs = e4m3x2(qd, 0.f) & 0xFFu;
+        const float rr = rtab[bs & 0x7Fu];  // p >= 0: bs is a non-negative code
 #pragma unroll
-        for (int e = 0; e < 16; ++e) p[e] = __fmul_rn(p[e], rr);
+        for (int e = 0; e < 16; e += 2) {
+          const float2 v = __fmul2_rn(make_float2(p[e], p[e + 1]), make_float2(rr, rr));
+          p[e] = v.x;
+          p[e + 1] = v.y;
+        }
         cw[2 * (cc & 1)] = e2m1x8(p);
         cw[2 * (cc & 1) + 1] = e2m1x8(p + 8);
         sfw |= bs << (8 * cc);
