@@ -499,6 +499,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         fail(abort_flag, a.err, kErrSoftmax);
       } else {
         tc_fence_after();
+        const float inv_l = __fdiv_rn(1.0f, l);
         const float* vs = a.v_scale + (size_t)bh * D + h * kHalfD;
         OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D + h * kHalfD;
 #pragma unroll 1
@@ -511,8 +512,8 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c = 32 * i + 2 * e;
-              hh[e] = pack2<OutT>(__fdiv_rn(__fmul_rn(u2f(o[2 * e]), __ldg(vs + c)), l),
-                                  __fdiv_rn(__fmul_rn(u2f(o[2 * e + 1]), __ldg(vs + c + 1)), l));
+              hh[e] = pack2<OutT>(div_by(__fmul_rn(u2f(o[2 * e]), __ldg(vs + c)), l, inv_l),
+                                  div_by(__fmul_rn(u2f(o[2 * e + 1]), __ldg(vs + c + 1)), l, inv_l));
             }
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)

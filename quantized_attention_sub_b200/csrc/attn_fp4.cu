@@ -530,6 +530,7 @@ __global__ void __launch_bounds__(kThreadsF, 2)
     } else {
       tc_fence_after();
       const float gpv = __fmul_rn(gp, gsc.z);
+      const float inv_l = __fdiv_rn(1.0f, l);
       OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D + h * 64;
 #pragma unroll 1
       for (int i = 0; i < 2; ++i) {
@@ -540,8 +541,8 @@ __global__ void __launch_bounds__(kThreadsF, 2)
           uint32_t hh[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            hh[e] = pack2<OutT>(__fdiv_rn(__fmul_rn(u2f(o[2 * e]), gpv), l),
-                                __fdiv_rn(__fmul_rn(u2f(o[2 * e + 1]), gpv), l));
+            hh[e] = pack2<OutT>(div_by(__fmul_rn(u2f(o[2 * e]), gpv), l, inv_l),
+                                div_by(__fmul_rn(u2f(o[2 * e + 1]), gpv), l, inv_l));
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             *reinterpret_cast<uint4*>(orow + 32 * i + 8 * v4) =

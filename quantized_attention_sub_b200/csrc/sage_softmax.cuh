@@ -85,6 +85,15 @@ SAGE_DEV float2 ex2_poly2(float2 d) {
   return make_float2(u2f(f2u(p.x) + (f2u(t.x) << 23)), u2f(f2u(p.y) + (f2u(t.y) << 23)));
 }
 
+// a / b from a correctly rounded reciprocal inv = RN(1/b): q = a * inv, then
+// one FMA correction (Markstein's division).  The correctly rounded quotient
+// while the residual a - b q does not underflow; a last-bit difference at
+// worst below that.
+SAGE_DEV float div_by(float a, float b, float inv) {
+  const float q = __fmul_rn(a, inv);
+  return __fmaf_rn(__fmaf_rn(-b, q, a), inv, q);
+}
+
 template <typename OutT>
 SAGE_DEV uint32_t pack2(float a, float b);
 template <>
