@@ -160,6 +160,7 @@ struct AttnF4Args {
   void* out;
   int* err;
   int N, Npad, causal;
+  int grouped;  // grid (G, query tiles, B*H/G) instead of (query tiles, B*H)
   float c_log2;
 };
 
@@ -191,8 +192,12 @@ __global__ void __launch_bounds__(kThreadsF, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_ktiles = a.Npad / 128;
-  const int qt = a.causal ? (n_ktiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int bh = blockIdx.y;
+  // Grid (query tiles, B*H): one slice's CTAs together (K and V in L2),
+  // causal tiles longest-first within the slice; grouped (G, query tiles,
+  // B*H/G): longest-first across G slices at a time (see causal_slice_group).
+  const int qi = a.grouped ? (int)blockIdx.y : (int)blockIdx.x;
+  const int qt = a.causal ? (n_ktiles - 1 - qi) : qi;
+  const int bh = a.grouped ? (int)(blockIdx.z * gridDim.x + blockIdx.x) : (int)blockIdx.y;
   const int T = a.causal ? qt + 1 : n_ktiles;
 
   if (threadIdx.x == 0) {
@@ -568,7 +573,10 @@ cudaError_t run_attn_fp4(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   auto kern = attn_fp4_kernel<OutT, HAS_BIAS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemF::alloc);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(ntiles, BH), kThreadsF, SmemF::alloc, s>>>(mq, mk, mv, a);
+  // packed K and V codes: 64 + 64 bytes per token of a slice
+  const int G = causal_slice_group(BH, 128.0 * a.Npad, 80e6);
+  const dim3 grid = a.grouped ? dim3(G, ntiles, BH / G) : dim3(ntiles, BH);
+  kern<<<grid, kThreadsF, SmemF::alloc, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -593,6 +601,9 @@ cudaError_t launch_attn_fp4(const WsPtrs& w, void* out, const Problem& pb, cudaS
   a.N = pb.N;
   a.Npad = pb.Npad;
   a.causal = pb.causal;
+  // causal: longest-first across slices when the longest CTA is a sizeable
+  // share of one SM's work (two CTAs per SM; as for the INT8/FP8 kernel)
+  a.grouped = pb.causal && (double)pb.BH * (pb.Npad / 128 + 1) < 11840.0;
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)pb.d));
   const int ntiles = pb.Npad / 128;
   const bool bias = a.bias != nullptr;

@@ -29,6 +29,17 @@ struct Problem {
   int BH, N, Npad, d, dtype, smooth_q, mode, causal;
 };
 
+// Causal attention grids run (G, query blocks, B*H/G): the CTAs of G slices
+// launch longest-first together, then the next G.  G is the largest divisor
+// of B*H whose K and V codes (slice_bytes each) fit in `budget` bytes of L2,
+// at least 1.
+inline int causal_slice_group(int BH, double slice_bytes, double budget) {
+  int g = 1;
+  for (int c = 1; c <= BH; ++c)
+    if (BH % c == 0 && c * slice_bytes <= budget) g = c;
+  return g;
+}
+
 // Launch `kern` on `s`; with `pdl` it may start while the previous kernel on
 // the stream is still running (programmatic stream serialization): the kernel
 // must call grid_dep_wait before it reads what that kernel wrote.
