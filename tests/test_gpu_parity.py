@@ -212,13 +212,13 @@ def test_full_size_video_dit_sampled_rows():
     compare_out(got, ref, "fp16", "video_dit")
 
 
-@pytest.mark.parametrize("N,d,causal", [(8192, 128, False), (2048, 64, True), (16384, 64, True)])
+@pytest.mark.parametrize("N,d,causal", [(8192, 128, False), (2048, 64, True), (8192, 64, True), (16384, 64, True)])
 def test_sweep_points_sampled_rows(N, d, causal):
     """Points of the kernel-speed sweep (B4 H32 fp16, K bias N(0, 2^2)):
     quantization bit-exact everywhere, the output on sampled rows of every
-    head (tile edges, the last row, random rows).  The two causal points
-    launch in the two causal CTA orders (longest-first across slices at
-    N 2048, per slice at N 16384)."""
+    head (tile edges, the last row, random rows).  The causal points cover
+    the causal CTA orders: longest-first across all 128 slices (N 2048), in
+    two groups of 64 slices (N 8192), and per slice (N 16384)."""
     w = inputs.sweep(N, d, causal)
     B, H = w.B, w.H
     q, k, v = [t.cuda() for t in inputs.generate(w)]
