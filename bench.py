@@ -50,7 +50,7 @@ FP4_OVER_BF16 = 4.0   # nominal dense ratio 9 / 2.25 PFLOP/s
 # size, from one ncu capture of the kernel as it stands on a smaller case
 # (inputs still above L2), scaled by the token count (attention traffic is
 # the codes read once plus the output, linear in N).  null for other sizes.
-TRAFFIC_BYTES = {"llm_prefill": 131.4e6, "video_dit": 196.3e6, "nvfp4": 66.8e6}
+TRAFFIC_BYTES = {"llm_prefill": 129.9e6, "video_dit": 200.6e6, "nvfp4": 66.8e6}
 
 # per mode: tensor peak ratio to bf16, attention kernel, arithmetic description
 MODE_INFO = {

@@ -130,8 +130,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   // K and V in L2; causal blocks launch longest-first within the slice.
   // Grouped (causal, few CTAs per SM): (G, query blocks, B*H/G), the blocks of
   // G slices longest-first across those slices (see causal_slice_group).
-  const int qi = a.grouped ? (int)blockIdx.y : (int)blockIdx.x;
-  const int qb = a.causal ? (a.num_qblocks - 1 - qi) : qi;
+  // (written so that the slice and block indices rematerialize cheaply: a
+  // variant that kept them live spilled registers and ran 2 % slower)
+  const int qb = a.causal ? (a.num_qblocks - 1 - (int)(a.grouped ? blockIdx.y : blockIdx.x)) : (int)blockIdx.x;
   const int bh = a.grouped ? (int)(blockIdx.z * gridDim.x + blockIdx.x) : (int)blockIdx.y;
   const int n_ktiles = a.Npad / 128;
   int nt[kNQ];
@@ -340,12 +341,16 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           lim = min(lim, a.N - kbase);
           if (a.causal) lim = min(lim, row - kbase + 1);
         }
-        // the tile's 64 bias values, loaded before the wait for S hides their latency
-        float4 bv[HAS_BIAS ? 16 : 1];
+        // FP16 mode: the tile's 64 bias values, loaded before the wait for S
+        // hides their latency (measured faster than loading half of them ahead,
+        // despite a few spilled registers); the FP32 mode, whose 576 threads
+        // leave no registers for it, loads them where they are used
+        constexpr int kAhead = F16ACC ? 16 : 0;
+        float4 bv[HAS_BIAS && kAhead > 0 ? kAhead : 1];
         if (HAS_BIAS) {
           const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4) bv[c4] = __ldg(b4 + c4);
+          for (int c4 = 0; c4 < kAhead; ++c4) bv[c4] = __ldg(b4 + c4);
         }
         // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
         if (!__all_sync(0xffffffffu, mbar_wait(&s_full[q], j & 1, abort_flag))) {
@@ -390,13 +395,15 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         } else {
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
           float ma = -INFINITY, mb = -INFINITY;
+          const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
             const int c = 4 * c4;
+            const float4 bw = c4 < kAhead ? bv[c4 < kAhead ? c4 : 0] : __ldg(b4 + c4);
             const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
-                                         __fmul2_rn(make_float2(bv[c4].x, bv[c4].y), cl2));
+                                         __fmul2_rn(make_float2(bw.x, bw.y), cl2));
             const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf),
-                                         __fmul2_rn(make_float2(bv[c4].z, bv[c4].w), cl2));
+                                         __fmul2_rn(make_float2(bw.z, bw.w), cl2));
             sr[c] = f2u(ta.x);
             sr[c + 1] = f2u(ta.y);
             sr[c + 2] = f2u(tb.x);
