@@ -46,11 +46,6 @@ SAGE_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-// Raise the phase's expected transaction bytes without arriving.
-SAGE_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
 SAGE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -128,15 +123,6 @@ SAGE_DEV bool named_bar_and(int id, int n, bool pred) {
       : "r"((uint32_t)pred), "r"(id), "r"(n)
       : "memory");
   return r != 0;
-}
-// Orders this thread's earlier generic-proxy view of global memory before its
-// later async-proxy (bulk copy) reads of it.
-SAGE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-// Acquire load of a flag written with release semantics by another CTA.
-SAGE_DEV int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
 }
 // Packed pairs of fp32 (each lane IEEE round-to-nearest, no flush to zero).
 // ptxas may contract mul2 followed by add2 into one fused multiply-add even
