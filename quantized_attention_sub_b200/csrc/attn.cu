@@ -1,10 +1,13 @@
 // attn.cu -- fused quantized attention forward for sm_100a, INT8 QK^T and FP8
 // P~V with an FP32 accumulator (SageAttention2 abstract; SageAttention2++
 // summary Sec. 2, 2.1: FlashAttention-based, per-block Q/K scales, per-channel
-// V scale, rescale at the end).
+// V scale, rescale at the end), and the same kernel with the FP16 P~V
+// accumulator of SageAttention2++ Sec. 3 (F16ACC: one query tile per CTA,
+// 320 threads, the 64-key f16 chunk partials folded into the fp32 row).
 //
 // One CTA owns two 128-query tiles of one (b, h) slice and walks the key
-// tiles of 128 in order.  Warp roles (576 threads, 18 warps):
+// tiles of 128 in order (causal: the longest query blocks launch first, see
+// the grid mapping in the kernel).  Warp roles (576 threads, 18 warps):
 //   warps 0-15  softmax: warpgroup g = warp / 4 handles query tile q = g / 2
 //               and key half h = g % 2 (keys [64h, 64h + 64) of every tile,
 //               one 64-key scale granule); thread <-> row <-> TMEM lane.
@@ -22,10 +25,12 @@
 //   wait for the previous P~V, multiply their half of the O row by alpha
 //   (skipped when alpha == 1 on the whole warp), write their 64 P~ bytes into
 //   the 128B-swizzled K-major shared tile the MMA reads, l_h = alpha l_h + sum p'.
-// At the end l = l_0 + l_1 and O = acc * scale_v / l is cast and stored.
-// exp2 runs on the special-function unit (ex2.approx); the CPU reference
-// computation uses the library exp2, so a P~ code may differ in rare cases and
-// the output is compared within a tolerance.
+// At the end l = l_0 + l_1 and O = acc * scale_v / l is cast and stored (the
+// quotient through one reciprocal of l per row and an FMA correction).
+// exp2 runs on the special-function unit (ex2.approx; in the FP16 mode a
+// quarter on a polynomial, ex2_poly2); the CPU reference computation uses the
+// library exp2, so a P~ code may differ in rare cases and the output is
+// compared within a tolerance.
 // Every wait is bounded (sage_ptx.cuh); a timeout records an error code in
 // the workspace, makes the other roles stop, and the CTA frees its TMEM.
 #include <cuda_bf16.h>

@@ -120,11 +120,13 @@ __global__ void __launch_bounds__(128)
 //   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
 //   p = exp2(t - m_new) on the special-function unit (the argument in the
 //   INT8 mode's steps), l_h = alpha l_h + sum p,
-//   per 16 keys: bs = ue4m3(max p / (6 g_p)), r = 1 / (g_p dec(bs)),
+//   per 16 keys: bs = ue4m3(max p / (6 g_p)) (an FMA-corrected quotient),
+//   r = 1 / (g_p dec(bs)) (from a table of the 128 scale codes),
 //   P~ = e2m1(p r): 32 bytes of codes into the 64-byte swizzled P~ row and
 //   one 32-bit word of four scales into TMEM (tcgen05.st),
 //   wait for the previous P~V, multiply their half of the O row by alpha.
-// At the end l = l_0 + l_1 and O = acc * (g_p g_v) / l.
+// At the end l = l_0 + l_1 and O = acc * (g_p g_v) / l (one reciprocal of l
+// per row and an FMA correction per output).
 // Every wait is bounded; a timeout records an error code in the workspace,
 // makes the other roles stop, and the CTA frees its TMEM.
 constexpr int kStagesF = 3;
