@@ -12,7 +12,7 @@ L2, so no flush runs between steps.
 Prints ONE JSON line (rank 0).  `value` is whole-job attention TOPS,
 4*B*H*N^2*d per step over the step time (the workload's metric, causal runs
 included); `value_executed` counts only the (query, key) pairs the mask
-leaves visible (causal: N(N+1)/2 per row block), the work the kernel does,
+leaves visible (causal: N(N+1)/2 pairs per slice), the work the kernel does,
 and the roofline fractions use that count.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
