@@ -205,7 +205,7 @@ ORC_EXPORT void orc_channel_absmax(const float* x, int BH, int N, int d, float* 
 
 /* ------------------------------------------------------------------------ */
 /* INT8 quantization of Q and K (SageAttention2++ Sec. 2.1: per-block scale   */
-/* factors; the spec granule reading: Q 32 tokens, K 64 tokens).        */
+/* factors; granules read as Q 32 tokens, K 64 tokens).                      */
 /* ------------------------------------------------------------------------ */
 
 /* x~ = x - mean (mean may be NULL: no smoothing).  Per granule of G tokens

@@ -235,7 +235,7 @@ def _small(N, d=64, H=2, dtype="fp16", seed=1001, law="k_bias", causal=False, sm
 @pytest.mark.parametrize("mode", [orc.MODE_INT8_FP8, orc.MODE_INT8_FP8_F16ACC])
 @pytest.mark.parametrize("causal", [False, True])
 def test_quantized_attention_close_to_fp64(mode, causal):
-    """North-star oracle check: cos >= 0.999 against unquantized fp64 attention."""
+    """Oracle accuracy check: cos >= 0.999 against unquantized fp64 attention."""
     w, q, k, v = _small(128)
     qz = orc.quantize_int8_fp8(q, k, v, smooth_q=False, mode=mode)
     o = orc.attention_int8_fp8(qz, causal)
