@@ -147,7 +147,11 @@ SAGE_API sage_status sage_quantize_qkv_static(const void* q, const void* k, cons
  * QK^T on the tensor cores, dequantize (scale_q * scale_k, plus the Q bias),
  * online softmax in base 2, P~ = e4m3(p * Pr) with Pr = 448 (224 in the F16ACC
  * mode), FP8 P~ V, and O = acc * scale_v / (Pr * l) (SageAttention2++ Sec. 2,
- * 2.1, 3).  causal masks key j > query i.  out: device [B,H,N,d] of `dtype`. */
+ * 2.1, 3).  SAGE_MODE_NVFP4 (SageAttention3 abstract): block-scaled e2m1 QK^T
+ * and P~ V (tcgen05 kind::mxf4nvf4), P~ quantized per 16 keys with ue4m3
+ * scales and global scale 1/(6*448); d must be 128 (SAGE_ERR_UNSUPPORTED
+ * otherwise).  causal masks key j > query i.  out: device [B,H,N,d] of
+ * `dtype`. */
 SAGE_API sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
                                 int causal, int smooth_q, int mode, sage_stream_t stream);
 
