@@ -16,9 +16,11 @@ the fp16/bf16 tensors both sides consume.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
+import tempfile
 
 import numpy as np
 
@@ -39,38 +41,80 @@ MODE_INT8_FP8, MODE_INT8_FP8_F16ACC, MODE_NVFP4 = 0, 1, 2
 _lib = None
 
 
+def _compile(src: str, out: str) -> None:
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+                           "-fPIC", "-shared", "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+
+
 def build(force: bool = False) -> str:
     """Compile sage_oracle.c into libsage_oracle.so (gcc, OpenMP, no FMA contraction)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-                               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
+        _compile(_SRC, _LIB)
     return _LIB
+
+
+def build_variant(edits) -> str:
+    """Compile a copy of sage_oracle.c with textual edits [(old, new), ...]
+    applied (each `old` must occur exactly once) into a temporary library and
+    return its path.  Used by the tests that plant a mistake in the oracle and
+    check that a pin catches it; the product never calls it."""
+    src = open(_SRC).read()
+    for old, new in edits:
+        n = src.count(old)
+        if n != 1:
+            raise ValueError("edit target found %d times: %r" % (n, old[:60]))
+        src = src.replace(old, new)
+    d = tempfile.mkdtemp(prefix="orc_variant_")
+    path = os.path.join(d, "sage_oracle_variant.c")
+    with open(path, "w") as f:
+        f.write(src)
+    out = os.path.join(d, "libsage_oracle_variant.so")
+    _compile(path, out)
+    return out
+
+
+@contextlib.contextmanager
+def using(path: str):
+    """Run the wrappers of this module against another build of the oracle
+    (a variant from build_variant) inside the `with` block."""
+    global _lib
+    saved = lib()
+    _lib = _declare(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    L.orc_e4m3_decode.restype = ctypes.c_double
+    L.orc_e4m3_decode.argtypes = [ctypes.c_int]
+    L.orc_e4m3_encode.restype = ctypes.c_int
+    L.orc_e4m3_encode.argtypes = [ctypes.c_double]
+    L.orc_ue4m3_encode.restype = ctypes.c_int
+    L.orc_ue4m3_encode.argtypes = [ctypes.c_double]
+    L.orc_ue4m3_decode.restype = ctypes.c_double
+    L.orc_ue4m3_decode.argtypes = [ctypes.c_int]
+    L.orc_e2m1_encode.restype = ctypes.c_int
+    L.orc_e2m1_encode.argtypes = [ctypes.c_double]
+    L.orc_e2m1_decode.restype = ctypes.c_double
+    L.orc_e2m1_decode.argtypes = [ctypes.c_int]
+    L.orc_f16_round.restype = ctypes.c_double
+    L.orc_f16_round.argtypes = [ctypes.c_double]
+    L.orc_num_threads.restype = ctypes.c_int
+    L.orc_exp2.restype = ctypes.c_float
+    L.orc_exp2.argtypes = [ctypes.c_float]
+    L.orc_nvfp4_block.restype = ctypes.c_int
+    L.orc_nvfp4_block.argtypes = [ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p]
+    return L
 
 
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
-        L = _lib
-        L.orc_e4m3_decode.restype = ctypes.c_double
-        L.orc_e4m3_decode.argtypes = [ctypes.c_int]
-        L.orc_e4m3_encode.restype = ctypes.c_int
-        L.orc_e4m3_encode.argtypes = [ctypes.c_double]
-        L.orc_ue4m3_encode.restype = ctypes.c_int
-        L.orc_ue4m3_encode.argtypes = [ctypes.c_double]
-        L.orc_ue4m3_decode.restype = ctypes.c_double
-        L.orc_ue4m3_decode.argtypes = [ctypes.c_int]
-        L.orc_e2m1_encode.restype = ctypes.c_int
-        L.orc_e2m1_encode.argtypes = [ctypes.c_double]
-        L.orc_e2m1_decode.restype = ctypes.c_double
-        L.orc_e2m1_decode.argtypes = [ctypes.c_int]
-        L.orc_f16_round.restype = ctypes.c_double
-        L.orc_f16_round.argtypes = [ctypes.c_double]
-        L.orc_num_threads.restype = ctypes.c_int
-        L.orc_exp2.restype = ctypes.c_float
-        L.orc_exp2.argtypes = [ctypes.c_float]
+        _lib = _declare(ctypes.CDLL(build()))
     return _lib
 
 
@@ -206,10 +250,12 @@ def quantize_int8_fp8(q, k, v, smooth_q: bool, mode: int) -> dict:
                 N=q.shape[1], d=q.shape[2], mode=mode)
 
 
-def attention_int8_fp8(qz: dict, causal: bool, rows=None) -> np.ndarray:
+def attention_int8_fp8(qz: dict, causal: bool, rows=None, with_flip: bool = False):
     """Tiled online-softmax attention on quantized inputs.  rows: None (all)
     or an int array of query rows (same rows for every slice).
-    Returns float32 [BH, nrows, d] before the cast to the output dtype."""
+    Returns float32 [BH, nrows, d] before the cast to the output dtype; with
+    `with_flip`, also the per-element change one P~ code moved to a
+    neighbouring code would cause (a sensitivity figure for comparisons)."""
     qc, kc, vt = qz["q_codes"], qz["k_codes"], qz["vt_codes"]
     BH, Np, d = qc.shape
     N = qz["N"]
@@ -222,11 +268,12 @@ def attention_int8_fp8(qz: dict, causal: bool, rows=None) -> np.ndarray:
         r = np.ascontiguousarray(rows, np.int32)
         nrows = len(r)
     out = np.empty((BH, nrows, d), np.float32)
+    flip = np.empty((BH, nrows, d), np.float32) if with_flip else None
     bias = qz["q_bias"]
     lib().orc_attn_int8_fp8(_p(qc), _p(qz["q_scale"]), _p(kc), _p(qz["k_scale"]), _p(vt),
                             _p(qz["v_scale"]), _p(bias), BH, N, Np, d, int(causal), int(mode),
-                            ctypes.c_float(Pr), _p(r), nrows, _p(out))
-    return out
+                            ctypes.c_float(qz.get("Pr", Pr)), _p(r), nrows, _p(out), _p(flip))
+    return (out, flip) if with_flip else out
 
 
 # --------------------------------------------------------------------------
@@ -259,7 +306,8 @@ def quantize_nvfp4(q, k, v, smooth_q: bool) -> dict:
     return out
 
 
-def attention_nvfp4(qz: dict, causal: bool, rows=None) -> np.ndarray:
+def attention_nvfp4(qz: dict, causal: bool, rows=None, with_flip: bool = False):
+    """NVFP4 attention (see attention_int8_fp8 for rows and with_flip)."""
     BH, Np, d = qz["q_codes"].shape
     N = qz["N"]
     if rows is None:
@@ -268,11 +316,21 @@ def attention_nvfp4(qz: dict, causal: bool, rows=None) -> np.ndarray:
         r = np.ascontiguousarray(rows, np.int32)
         nrows = len(r)
     out = np.empty((BH, nrows, d), np.float32)
+    flip = np.empty((BH, nrows, d), np.float32) if with_flip else None
     lib().orc_attn_nvfp4(_p(qz["q_codes"]), _p(qz["q_bscale"]), _p(qz["q_gscale"]),
                          _p(qz["k_codes"]), _p(qz["k_bscale"]), _p(qz["k_gscale"]),
                          _p(qz["vt_codes"]), _p(qz["vt_bscale"]), _p(qz["v_gscale"]),
-                         _p(qz["q_bias"]), BH, N, Np, d, int(causal), _p(r), nrows, _p(out))
-    return out
+                         _p(qz["q_bias"]), BH, N, Np, d, int(causal), _p(r), nrows, _p(out), _p(flip))
+    return (out, flip) if with_flip else out
+
+
+def nvfp4_block(x, g: float):
+    """The NVFP4 block quantizer on 16 values with global scale g: returns
+    (ue4m3 scale code, 16 e2m1 codes)."""
+    x = _f32(np.asarray(x).reshape(16))
+    codes = np.empty(16, np.uint8)
+    bs = lib().orc_nvfp4_block(_p(x), ctypes.c_float(g), _p(codes))
+    return bs, codes
 
 
 # --------------------------------------------------------------------------

@@ -22,10 +22,14 @@
  *   - SageAttention3 abstract: microscaling FP4 attention (NVFP4 mode).
  * Where the pages are silent the readings are written next to each function.
  *
- * Arithmetic: IEEE binary32 round-to-nearest-even for every step the kernels
- * take in fp32 (compiled with -ffp-contract=off, no fast-math; an FMA only
- * where fmaf is written).  Sums the pages leave unspecified are exact (double
- * holds them exactly, see each comment).
+ * Arithmetic: IEEE binary32 round-to-nearest-even, one rounding per written
+ * operation (compiled with -ffp-contract=off, no fast-math; an FMA only where
+ * fmaf is written).  The pages fix the formats of the quantized operands (INT8,
+ * FP8, FP4, the FP16 accumulator) but no precision for the statistics and the
+ * softmax; those steps are taken in fp32, the precision in which every
+ * quantized code is decided, in the order the method states them.  Sums the
+ * pages leave unspecified are exact (double holds them exactly, see each
+ * comment).
  *
  * Layouts (all row-major, contiguous):
  *   x        [BH, N, d]        input (already converted to float)
@@ -153,11 +157,8 @@ ORC_EXPORT double orc_f16_round(double x)
   return x < 0 ? -r : r;
 }
 
-/* exp2 of the softmax: the library exp2 in double, rounded once to fp32.
- * The pages fix no accuracy for the exponential; the GPU evaluates it on its
- * special-function unit (ex2.approx), whose result may differ from this one
- * in the last bits, so a P~ code can differ in rare cases and the attention
- * output is compared within a tolerance.  -inf gives +0. */
+/* exp2 of the softmax: the library exp2 in double, rounded once to fp32
+ * (the pages fix no accuracy for the exponential).  -inf gives +0. */
 ORC_EXPORT float orc_exp2(float d)
 {
   return (float)exp2((double)d);
@@ -321,34 +322,48 @@ ORC_EXPORT void orc_qk_s32(const int8_t* q, const int8_t* k, int nq, int nk, int
 
 enum { ORC_MODE_FP32ACC = 0, ORC_MODE_F16ACC = 1 };
 
+/* Distance from e4m3 magnitude code cm to its farther neighbour: the most a
+ * P~ value moves when its code lands one step away. */
+static double e4m3_step(int cm)
+{
+  double v = g_e4m3_mag[cm];
+  double up = cm < 126 ? g_e4m3_mag[cm + 1] - v : 0.0;
+  double dn = cm > 0 ? v - g_e4m3_mag[cm - 1] : 0.0;
+  return up > dn ? up : dn;
+}
+
 /* One query row, FlashAttention order: key tiles of 128 in ascending order.
- * Per tile (only tiles holding at least one key the row may see):
- *   kf    = (sq_i * sk_g(j)) * (log2(e) / sqrt(d))        one factor per 64-key granule
- *   t_j   = float(S_ij) * kf, or fma(float(S_ij), kf, bias_j * (log2(e)/sqrt(d)))
- *   m_new = max(m, max_j t_j);  alpha = exp2(m - m_new);  m' = m_new - log2(Pr)
- *   p'_j  = exp2(d_j) = p_j * Pr with p_j the softmax numerator, where
- *           d_j = fma(float(S_ij), kf, -m') in one rounding (t_j - m' with a
- *           bias);
- *   l     = alpha * l + sum_j p'_j        (in units of Pr)
- *   P~_j  = e4m3(p'_j)
+ * Per tile (only tiles holding at least one key the row may see), in fp32:
+ *   t_j   = ((float(S_ij) * (sq_i * sk_g(j))) + bias_j) * (log2(e) / sqrt(d))
+ *           (the dequantized score plus the Q-smoothing bias, in base-2 units;
+ *           without Q smoothing there is no bias term)
+ *   m_new = max(m, max_j t_j);  alpha = exp2(m - m_new)
+ *   p_j   = exp2(t_j - m_new)                  (p <= 1)
+ *   l     = alpha * l + sum_j p_j              (sequential fp32 sum)
+ *   P~_j  = e4m3(p_j * Pr)                     (static P~ scale 1/Pr)
  *   FP32 accumulator: acc_c = alpha * acc_c + fl32(exact sum_j P~_j v^_jc)
  *   FP16 accumulator (SageAttention2++ Sec. 3.2): per 64-key chunk,
  *        h = f16(exact sum of its first 32 products), h = f16(h + exact sum of
- *        the next 32); acc_c = alpha * acc_c + h_chunk0 + h_chunk1
- *   O_ic  = acc_c * scale_v[c] / l
+ *        the next 32); acc_c = (alpha * acc_c + h_chunk0) + h_chunk1
+ *   O_ic  = acc_c * scale_v[c] / (Pr * l)
  * exp2 is orc_exp2 above.  Masked keys (j >= N, or j > i when causal) take no
  * part.  The exact sums of e4m3 products fit a double: each product has 8
  * significant bits within 2^-18..2^18 and at most 128 are added.
- * out_row receives fp32 results (the caller rounds to the output dtype). */
+ * out_row receives fp32 results (the caller rounds to the output dtype).
+ * flip_row (may be NULL) receives, per channel, the largest change of O_ic
+ * that moving one P~ code of the row to a neighbouring code would cause:
+ * max over keys of step(P~_j) * |v^_jc| carried through the later rescales,
+ * times scale_v[c] / (Pr * l).  It is a sensitivity figure for comparisons
+ * with implementations whose exponential differs in the last bits. */
 static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* vt,
                      float sq, const float* sk, const float* bias, const float* scale_v,
                      int N, int Npad, int d, int causal, int mode, float Pr,
-                     float* acc, float* tvals, float* xvals, int* pcode, float* out_row)
+                     float* acc, double* fl, float* tvals, int* pcode, float* out_row,
+                     float* flip_row)
 {
   const float c_log2 = (float)(1.4426950408889634 / sqrt((double)d));
-  const float log2Pr = (float)log2((double)Pr);
   float m = -INFINITY, l = 0.0f;
-  for (int c = 0; c < d; ++c) acc[c] = 0.0f;
+  for (int c = 0; c < d; ++c) { acc[c] = 0.0f; fl[c] = 0.0; }
   int jmax = causal ? (i < N - 1 ? i : N - 1) : N - 1;   /* last visible key */
   for (int j0 = 0; j0 <= jmax; j0 += 128) {
     float mt = -INFINITY;
@@ -356,41 +371,44 @@ static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* v
       if (j > jmax) { tvals[j - j0] = -INFINITY; continue; }
       int32_t s = 0;
       for (int c = 0; c < d; ++c) s += (int32_t)qc[(size_t)i * d + c] * (int32_t)kc[(size_t)j * d + c];
-      const float x = (float)s;
-      const float kf = (sq * sk[j / 64]) * c_log2;
-      const float t = bias ? fmaf(x, kf, bias[j] * c_log2) : x * kf;
-      xvals[j - j0] = x;
+      float deq = (float)s * (sq * sk[j / 64]);
+      if (bias) deq = deq + bias[j];
+      const float t = deq * c_log2;
       tvals[j - j0] = t;
       if (t > mt) mt = t;
     }
     const float m_new = m > mt ? m : mt;
     const float alpha = orc_exp2(m - m_new);   /* first tile: exp2(-inf) = 0 */
-    const float mp = m_new - log2Pr;
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
       float p = 0.0f;
-      if (j0 + j <= jmax) {
-        /* d = t - m' (without bias in one rounding: fma(x, kf, -m')) */
-        const float kf = (sq * sk[(j0 + j) / 64]) * c_log2;
-        const float dd = bias ? tvals[j] - mp : fmaf(xvals[j], kf, -mp);
-        p = orc_exp2(dd);
-      }
+      if (j0 + j <= jmax) p = orc_exp2(tvals[j] - m_new);
       ps = ps + p;
-      pcode[j] = orc_e4m3_encode((double)p);
+      pcode[j] = (j0 + j <= jmax) ? orc_e4m3_encode((double)(p * Pr)) : -1;
     }
     l = alpha * l + ps;
     for (int c = 0; c < d; ++c) {
       const uint8_t* vrow = vt + (size_t)c * Npad + j0;
+      double fmx = fl[c] * alpha;
+      for (int j = 0; j < 128; ++j) {
+        if (pcode[j] < 0) continue;
+        double e = e4m3_step(pcode[j] & 0x7F) * fabs(orc_e4m3_decode(vrow[j]));
+        if (e > fmx) fmx = e;
+      }
+      fl[c] = fmx;
       if (mode == ORC_MODE_FP32ACC) {
         double sum = 0.0;
-        for (int j = 0; j < 128; ++j) sum += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
+        for (int j = 0; j < 128; ++j)
+          if (pcode[j] >= 0) sum += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
         acc[c] = alpha * acc[c] + (float)sum;
       } else {
         float a = alpha * acc[c];
         for (int ch = 0; ch < 128; ch += 64) {
           double s0 = 0.0, s1 = 0.0;
-          for (int j = ch; j < ch + 32; ++j) s0 += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
-          for (int j = ch + 32; j < ch + 64; ++j) s1 += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
+          for (int j = ch; j < ch + 32; ++j)
+            if (pcode[j] >= 0) s0 += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
+          for (int j = ch + 32; j < ch + 64; ++j)
+            if (pcode[j] >= 0) s1 += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
           double h = orc_f16_round(s0);
           h = orc_f16_round(h + s1);
           a = a + (float)h;
@@ -400,35 +418,41 @@ static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* v
     }
     m = m_new;
   }
-  for (int c = 0; c < d; ++c) out_row[c] = acc[c] * scale_v[c] / l;
+  const float den = Pr * l;
+  for (int c = 0; c < d; ++c) {
+    out_row[c] = acc[c] * scale_v[c] / den;
+    if (flip_row) flip_row[c] = (float)(fl[c] * scale_v[c] / den);
+  }
 }
 
 /* Attention output for the listed query rows of every (b,h) slice.
- * rows == NULL means all N rows (then nrows must be N).  out: [BH, nrows, d]. */
+ * rows == NULL means all N rows (then nrows must be N).  out: [BH, nrows, d].
+ * flip (may be NULL): [BH, nrows, d] single-code sensitivity (see attn_row). */
 ORC_EXPORT void orc_attn_int8_fp8(const int8_t* qc, const float* sq, const int8_t* kc,
                                   const float* sk, const uint8_t* vt, const float* scale_v,
                                   const float* bias, int BH, int N, int Npad, int d,
                                   int causal, int mode, float Pr, const int* rows, int nrows,
-                                  float* out)
+                                  float* out, float* flip)
 {
   init_tables();
 #pragma omp parallel
   {
     float* acc = (float*)malloc(sizeof(float) * d);
+    double* fl = (double*)malloc(sizeof(double) * d);
     float* tv = (float*)malloc(sizeof(float) * 128);
-    float* xv = (float*)malloc(sizeof(float) * 128);
     int* pc = (int*)malloc(sizeof(int) * 128);
 #pragma omp for schedule(dynamic, 4) collapse(2)
     for (int bh = 0; bh < BH; ++bh)
       for (int r = 0; r < nrows; ++r) {
         int i = rows ? rows[r] : r;
+        const size_t o = ((size_t)bh * nrows + r) * d;
         attn_row(i, qc + (size_t)bh * Npad * d, kc + (size_t)bh * Npad * d,
                  vt + (size_t)bh * d * Npad, sq[(size_t)bh * (Npad / 32) + i / 32],
                  sk + (size_t)bh * (Npad / 64), bias ? bias + (size_t)bh * Npad : NULL,
-                 scale_v + (size_t)bh * d, N, Npad, d, causal, mode, Pr, acc, tv, xv, pc,
-                 out + ((size_t)bh * nrows + r) * d);
+                 scale_v + (size_t)bh * d, N, Npad, d, causal, mode, Pr, acc, fl, tv, pc,
+                 out + o, flip ? flip + o : NULL);
       }
-    free(acc); free(tv); free(xv); free(pc);
+    free(acc); free(fl); free(tv); free(pc);
   }
 }
 
@@ -455,6 +479,14 @@ static int fp4_block(const float* x, int st, float g, uint8_t* out)
   for (int k = 0; k < 16; ++k)
     out[k] = (uint8_t)((sd > 0.0f) ? orc_e2m1_encode((double)(x[k * st] * r)) : 0);
   return bs;
+}
+
+/* The block quantizer above for one block of 16 contiguous values: returns
+ * the ue4m3 scale code, writes the 16 e2m1 codes (one per byte). */
+ORC_EXPORT int orc_nvfp4_block(const float* x, float g, uint8_t* codes)
+{
+  init_tables();
+  return fp4_block(x, 1, g, codes);
 }
 
 /* Q or K in NVFP4: x~ = x - mean (mean may be NULL); g = A / (6 * 448) with A
@@ -517,26 +549,41 @@ ORC_EXPORT void orc_quant_nvfp4_vt(const float* v, int BH, int N, int Npad, int 
   }
 }
 
+/* e2m1 step at magnitude code cm: distance to the farther neighbour. */
+static double e2m1_step(int cm)
+{
+  double v = g_e2m1_mag[cm];
+  double up = cm < 7 ? g_e2m1_mag[cm + 1] - v : 0.0;
+  double dn = cm > 0 ? v - g_e2m1_mag[cm - 1] : 0.0;
+  return up > dn ? up : dn;
+}
+
 /* NVFP4 attention for one row.  x_ij = sum_c dq_ic dk_jc where the
  * dequantized values are code * dec(block scale) (exact products, summed in
- * double, rounded once to fp32); then the logits and online softmax of the
- * INT8 mode with kf = (g_q g_k) log2(e)/sqrt(d) in place of its per-granule
- * factor and no P~ range factor; P~ in NVFP4 along keys with the constant
- * global scale g_p = 1 / (6 * 448) (p <= 1); PV summed exactly per tile and
- * added in fp32; O = acc * g_p * g_v / l. */
+ * double, rounded once to fp32); then the steps of the INT8 mode with the
+ * slice global scales in place of the per-granule scales:
+ *   t_j = ((x_ij * (g_q * g_k)) + bias_j) * (log2(e) / sqrt(d)),
+ *   m_new, alpha, p_j = exp2(t_j - m_new), l = alpha * l + sum_j p_j;
+ * P~ in NVFP4 along keys: blocks of 16 keys, the block quantizer of Q/K/V
+ * with the constant global scale g_p = 1 / (6 * 448) (p <= 1); PV summed
+ * exactly per tile and added in fp32; O = acc * (g_p * g_v) / l.
+ * flip_row (may be NULL): per channel, the largest change of O_ic that moving
+ * every code of one P~ block by one e2m1 step, its scale by one ue4m3 step
+ * (1/8), would cause -- the same sensitivity figure as in attn_row. */
 static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq,
                            const uint8_t* kc, const uint8_t* ks, float gk,
                            const uint8_t* vc, const uint8_t* vs, float gv, const float* bias,
-                           int N, int Npad, int d, int causal, double* qd, float* acc,
-                           float* tvals, float* xvals, float* pvals, uint8_t* pcodes, uint8_t* pbs,
-                           float* out_row)
+                           int N, int Npad, int d, int causal, double* qd, float* acc, double* fl,
+                           float* tvals, float* pvals, uint8_t* pcodes, uint8_t* pbs,
+                           float* out_row, float* flip_row)
 {
   const float c_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   const float gp = 1.0f / (6.0f * 448.0f);
-  const float kf = (gq * gk) * c_log2;
+  const float gqk = gq * gk;
   float m = -INFINITY, l = 0.0f;
   for (int c = 0; c < d; ++c) {
     acc[c] = 0.0f;
+    fl[c] = 0.0;
     qd[c] = orc_e2m1_decode(qc[(size_t)i * d + c]) * orc_ue4m3_decode(qs[(size_t)i * (d / 16) + c / 16]);
   }
   int jmax = causal ? (i < N - 1 ? i : N - 1) : N - 1;
@@ -547,9 +594,9 @@ static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq
       double s = 0.0;
       for (int c = 0; c < d; ++c)
         s += qd[c] * orc_e2m1_decode(kc[(size_t)j * d + c]) * orc_ue4m3_decode(ks[(size_t)j * (d / 16) + c / 16]);
-      const float x = (float)s;
-      const float t = bias ? fmaf(x, kf, bias[j] * c_log2) : x * kf;
-      xvals[j - j0] = x;
+      float deq = (float)s * gqk;
+      if (bias) deq = deq + bias[j];
+      const float t = deq * c_log2;
       tvals[j - j0] = t;
       if (t > mt) mt = t;
     }
@@ -558,43 +605,51 @@ static void attn_row_nvfp4(int i, const uint8_t* qc, const uint8_t* qs, float gq
     float ps = 0.0f;
     for (int j = 0; j < 128; ++j) {
       float p = 0.0f;
-      if (j0 + j <= jmax) {
-        const float dd = bias ? tvals[j] - m_new : fmaf(xvals[j], kf, -m_new);
-        p = orc_exp2(dd);
-      }
+      if (j0 + j <= jmax) p = orc_exp2(tvals[j] - m_new);
       pvals[j] = p;
       ps = ps + p;
     }
     l = alpha * l + ps;
     for (int b = 0; b < 8; ++b) pbs[b] = (uint8_t)fp4_block(pvals + b * 16, 1, gp, pcodes + b * 16);
     for (int c = 0; c < d; ++c) {
-      double sum = 0.0;
-      for (int j = 0; j < 128; ++j) {
-        int t = j0 + j;
-        double pj = orc_e2m1_decode(pcodes[j]) * orc_ue4m3_decode(pbs[j / 16]);
-        double vj = orc_e2m1_decode(vc[(size_t)c * Npad + t]) * orc_ue4m3_decode(vs[(size_t)c * (Npad / 16) + t / 16]);
-        sum += pj * vj;
+      double sum = 0.0, fmx = fl[c] * alpha;
+      for (int b = 0; b < 8; ++b) {
+        double fb = 0.0;
+        for (int j = 16 * b; j < 16 * b + 16; ++j) {
+          int t = j0 + j;
+          if (t > jmax) continue;
+          double vj = orc_e2m1_decode(vc[(size_t)c * Npad + t]) * orc_ue4m3_decode(vs[(size_t)c * (Npad / 16) + t / 16]);
+          sum += orc_e2m1_decode(pcodes[j]) * orc_ue4m3_decode(pbs[b]) * vj;
+          fb += (e2m1_step(pcodes[j] & 7) + 0.125 * orc_e2m1_decode(pcodes[j] & 7)) * orc_ue4m3_decode(pbs[b]) *
+                fabs(vj);
+        }
+        if (fb > fmx) fmx = fb;
       }
+      fl[c] = fmx;
       acc[c] = alpha * acc[c] + (float)sum;
     }
     m = m_new;
   }
-  for (int c = 0; c < d; ++c) out_row[c] = acc[c] * (gp * gv) / l;
+  const float gpv = gp * gv;
+  for (int c = 0; c < d; ++c) {
+    out_row[c] = acc[c] * gpv / l;
+    if (flip_row) flip_row[c] = (float)(fl[c] * gpv / l);
+  }
 }
 
 ORC_EXPORT void orc_attn_nvfp4(const uint8_t* qc, const uint8_t* qs, const float* gq,
                                const uint8_t* kc, const uint8_t* ks, const float* gk,
                                const uint8_t* vc, const uint8_t* vs, const float* gv,
                                const float* bias, int BH, int N, int Npad, int d, int causal,
-                               const int* rows, int nrows, float* out)
+                               const int* rows, int nrows, float* out, float* flip)
 {
   init_tables();
 #pragma omp parallel
   {
     double* qd = (double*)malloc(sizeof(double) * d);
     float* acc = (float*)malloc(sizeof(float) * d);
+    double* fl = (double*)malloc(sizeof(double) * d);
     float* tv = (float*)malloc(sizeof(float) * 128);
-    float* xv = (float*)malloc(sizeof(float) * 128);
     float* pv = (float*)malloc(sizeof(float) * 128);
     uint8_t* pc = (uint8_t*)malloc(128);
     uint8_t pbs[8];
@@ -602,12 +657,13 @@ ORC_EXPORT void orc_attn_nvfp4(const uint8_t* qc, const uint8_t* qs, const float
     for (int bh = 0; bh < BH; ++bh)
       for (int r = 0; r < nrows; ++r) {
         int i = rows ? rows[r] : r;
+        const size_t o = ((size_t)bh * nrows + r) * d;
         attn_row_nvfp4(i, qc + (size_t)bh * Npad * d, qs + (size_t)bh * Npad * (d / 16), gq[bh],
                        kc + (size_t)bh * Npad * d, ks + (size_t)bh * Npad * (d / 16), gk[bh],
                        vc + (size_t)bh * d * Npad, vs + (size_t)bh * d * (Npad / 16), gv[bh],
-                       bias ? bias + (size_t)bh * Npad : NULL, N, Npad, d, causal, qd, acc, tv,
-                       xv, pv, pc, pbs, out + ((size_t)bh * nrows + r) * d);
+                       bias ? bias + (size_t)bh * Npad : NULL, N, Npad, d, causal, qd, acc, fl, tv,
+                       pv, pc, pbs, out + o, flip ? flip + o : NULL);
       }
-    free(qd); free(acc); free(tv); free(xv); free(pv); free(pc);
+    free(qd); free(acc); free(fl); free(tv); free(pv); free(pc);
   }
 }

@@ -267,8 +267,12 @@ def test_f16acc_same_accuracy_as_fp32acc():
 
 
 def test_dropping_the_rescale_is_caught():
-    """A planted mistake in the oracle's tile loop (alpha forced to 1) must fail
-    the fp64 check: with several tiles the running max grows on random data."""
+    """The online softmax over several tiles against a single global-max
+    softmax of the same codes (rows whose max sits in the first tile), and
+    the quantized attention against fp64 on random data, where the running
+    max grows across tiles.  tests/test_oracle_plants.py plants a dropped
+    rescale and a wrong K-scale granule in a copy of the oracle and checks
+    that this test rejects both."""
     w, q, k, v = _small(1024, d=64)
     ref = orc.attention_fp64(q, k, v, False)
     qz = orc.quantize_int8_fp8(q, k, v, False, 0)
@@ -293,10 +297,10 @@ def test_dropping_the_rescale_is_caught():
     ptil = np.vectorize(lambda x: orc.e4m3_decode(orc.e4m3_encode(x)))(np.float32(p * 448.0))
     vdq = np.stack([orc.e4m3_decode_array(qz2["vt_codes"][b, :, :N]).T for b in range(2)])
     o_plain = (ptil @ vdq) * qz2["v_scale"][:, None, :] / (448.0 * p.sum(axis=2, keepdims=True))
-    # exact 2^x here vs the oracle's polynomial (within 8.6e-5): the row sums
-    # differ by up to ~1e-4 relative and a P~ code may flip where p*448 sits
-    # that close to a rounding midpoint; a dropped rescale gives errors of the
-    # size of O itself
+    # fp64 logits and exponentials here against the oracle's fp32 steps: the
+    # row sums differ in the last bits and a P~ code may flip where p*448 sits
+    # that close to a rounding midpoint; a dropped rescale, or a wrong scale
+    # granule, gives errors of the size of O itself
     err = np.abs(o2[:, rows] - o_plain[:, rows])
     assert np.max(err) < 5e-3 and np.mean(err) < 3e-4
 
