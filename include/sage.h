@@ -151,7 +151,9 @@ SAGE_API sage_status sage_quantize_qkv_static(const void* q, const void* k, cons
  * and P~ V (tcgen05 kind::mxf4nvf4), P~ quantized per 16 keys with ue4m3
  * scales and global scale 1/(6*448); d must be 128 (SAGE_ERR_UNSUPPORTED
  * otherwise).  causal masks key j > query i.  out: device [B,H,N,d] of
- * `dtype`. */
+ * `dtype`.  ws_bytes: at least sage_ws_layout.scratch (the quantized region;
+ * the statistics scratch after it is not read), so the output buffer of
+ * sage_quantize_qkv_static serves as well. */
 SAGE_API sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
                                 int causal, int smooth_q, int mode, sage_stream_t stream);
 
@@ -164,7 +166,8 @@ SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, 
 /* Parity helper: the INT32 tile S = Q^ K^T of query tile `q_tile` and key tile
  * `k_tile` (128 x 128) of slice `bh`, computed by the same tensor-core path as
  * the attention kernel (kind::i8 MMA, accumulator in TMEM).  out: device
- * int32 [128, 128], row = query.  INT8 modes only. */
+ * int32 [128, 128], row = query.  INT8 modes only.  ws_bytes: at least
+ * sage_ws_layout.scratch, as for sage_attn_quantized. */
 SAGE_API sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,
                               int k_tile, int32_t* out, sage_stream_t stream);
 

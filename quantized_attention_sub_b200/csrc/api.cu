@@ -89,10 +89,13 @@ sage::WsPtrs resolve(void* ws, const sage_ws_layout& L) {
   return w;
 }
 
-sage_status check_ws(const void* ws, size_t ws_bytes, const sage_ws_layout& L) {
+// `need`: bytes the call touches -- L.total for the quantization pass (it
+// writes the statistics scratch), L.scratch for the calls that only read the
+// quantized region below it (attention, the debug tiles).
+sage_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
   if (!ws) return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null%s");
   if (((uintptr_t)ws) % kAlign) return set_err(SAGE_ERR_INVALID_ARG, "workspace must be 1024-byte aligned%s");
-  if (ws_bytes < L.total) return set_err(SAGE_ERR_INVALID_ARG, "workspace too small%s");
+  if (ws_bytes < need) return set_err(SAGE_ERR_INVALID_ARG, "workspace too small%s");
   return SAGE_OK;
 }
 
@@ -113,14 +116,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // initialized once, thread-safely (C++11 static initialization)
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
+      return (EncodeTiledFn)p;
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -167,7 +171,7 @@ sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int d
   if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
     return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
-  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, 0};
   const float Vr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 4.5f : 448.0f;
   if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
@@ -220,7 +224,7 @@ static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, in
   if (mode == SAGE_MODE_NVFP4 && d != 128)
     return set_err(SAGE_ERR_UNSUPPORTED, "the NVFP4 attention kernel needs d = 128%s");
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
-  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L.scratch)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
   if (!after_quantize &&
       (st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
@@ -258,7 +262,7 @@ sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int
   if (!out || bh < 0 || bh >= B * H || q_tile < 0 || q_tile >= ntiles || k_tile < 0 || k_tile >= ntiles)
     return set_err(SAGE_ERR_INVALID_ARG, "debug tile out of range%s");
   const sage_ws_layout L = layout_of(B, H, N, d, SAGE_MODE_INT8_FP8);
-  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L.scratch)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, ntiles * 128, d, 0, 0, 0, 0};
   if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
@@ -276,7 +280,7 @@ sage_status sage_debug_fp4_s(const void* ws, size_t ws_bytes, int B, int H, int 
   if (!out || bh < 0 || bh >= B * H || q_tile < 0 || q_tile >= ntiles || k_tile < 0 || k_tile >= ntiles)
     return set_err(SAGE_ERR_INVALID_ARG, "debug tile out of range%s");
   const sage_ws_layout L = layout_of(B, H, N, d, SAGE_MODE_NVFP4);
-  if ((st = check_ws(ws, ws_bytes, L)) != SAGE_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L.scratch)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, ntiles * 128, d, 0, 0, SAGE_MODE_NVFP4, 0};
   if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;

@@ -649,12 +649,10 @@ static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const 
                             int BH, cudaStream_t s) {
   auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS, F16ACC>;
   using L = Smem<D, Roles<F16ACC>::kNQ>;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  // set on every launch: the attribute is per device, and a cached flag would
+  // be shared by host threads and devices
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
+  if (e != cudaSuccess) return e;
   const int G = causal_slice_group(BH, 2.0 * a.Npad * D, 80e6);
   const dim3 grid = a.grouped ? dim3(G, a.num_qblocks, BH / G) : dim3(a.num_qblocks, BH);
   kern<<<grid, Roles<F16ACC>::kThreads, L::alloc, s>>>(mq, mk, mv, a);

@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import oracle as orc
+from parity_check import compare_out
 from quantized_attention_sub_b200 import api, inputs
 
 pytestmark = pytest.mark.gpu
@@ -169,7 +170,6 @@ def test_nvfp4_attention_matches_oracle(N, dtype, law, smooth_q, causal):
     """The fused kind::mxf4nvf4 attention against the oracle's NVFP4
     attention on the same (bit-identical) codes and scales, output rounded to
     the dtype, with the INT8/FP8 modes' bounds."""
-    from test_gpu_parity import compare_out, to_dtype_np
     w = inputs.variant(inputs.WORKLOADS["unit"], N=N, d=128, H=2, dtype=dtype, law=law, smooth_q=smooth_q,
                        mode=api.MODE_NVFP4, causal=causal, seed=7300 + N)
     q, k, v = [t.cuda() for t in inputs.generate(w)]
@@ -179,9 +179,9 @@ def test_nvfp4_attention_matches_oracle(N, dtype, law, smooth_q, causal):
     api.sage_attn_fwd(q, k, v, out, B, H, N, d, causal, api.MODE_NVFP4, api.DTYPE_CODE[q.dtype], smooth_q, ws,
                       ws.numel())
     api.sage_check(ws, ws.numel())
-    ref = to_dtype_np(orc.attention_nvfp4(oracle_fp4(q, k, v, smooth_q), causal), dtype)
+    ref32, flip = orc.attention_nvfp4(oracle_fp4(q, k, v, smooth_q), causal, with_flip=True)
     got = out.float().cpu().reshape(B * H, N, d).numpy()
-    compare_out(got, ref, dtype, (N, dtype, law, smooth_q, causal))
+    compare_out(got, ref32, flip, dtype, (N, dtype, law, smooth_q, causal))
 
 
 def test_nvfp4_attention_rejects_d64():
@@ -197,7 +197,6 @@ def test_full_size_nvfp4_sampled_rows():
     """The B1 H16 N16384 d128 bf16 NVFP4 workload at full size, in the launch
     configuration the bench times: quantization bit-exact everywhere, the
     output on sampled rows per head (first, tile edges, last, random)."""
-    from test_gpu_parity import compare_out, to_dtype_np
     w = inputs.WORKLOADS["nvfp4"]
     B, H, N, d = w.shape()
     q, k, v = [t.cuda() for t in inputs.generate(w)]
@@ -211,6 +210,6 @@ def test_full_size_nvfp4_sampled_rows():
     assert_fp4_bitexact(g, oz, d, w.smooth_q)
     rng = np.random.default_rng(16384)
     rows = np.unique(np.concatenate([[0, 127, 128, N - 129, N - 1], rng.integers(0, N, 11)])).astype(np.int32)
-    ref = to_dtype_np(orc.attention_nvfp4(oz, w.causal, rows=rows), w.dtype)
+    ref32, flip = orc.attention_nvfp4(oz, w.causal, rows=rows, with_flip=True)
     got = out.float().cpu().reshape(B * H, N, d).numpy()[:, rows]
-    compare_out(got, ref, w.dtype, "nvfp4 full size")
+    compare_out(got, ref32, flip, w.dtype, "nvfp4 full size")
