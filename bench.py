@@ -5,15 +5,24 @@ One step = one pass of the whole hot path over one batch: smoothing + INT8/FP8
 quantization of Q, K, V (libsage quantize kernels) and the fused attention
 kernel, all through the C ABI (libsage.so).
 
-Default workload: LLM prefill, B1 H32 N8192 d128 bf16, causal, INT8 QK / FP8 PV
-(FP32 accumulator).  Inputs (192 MB of bf16 Q, K, V) are larger than the 126 MB
-L2, so no flush runs between steps.
+Headline workload: the kernel-speed sweep's target point, B4 H32 N32768 d128
+fp16, non-causal, INT8 QK / FP8 PV with the FP32 accumulator (the point the
+kernel's roofline aim is quoted on: N >= 16K, d = 128).  Its inputs (3 x 1.07
+GB) are far larger than the 126 MB L2, so no flush runs between steps.
 
 Prints ONE JSON line (rank 0).  `value` is whole-job attention TOPS,
-4*B*H*N^2*d per step over the step time (the workload's metric, causal runs
-included); `value_executed` counts only the (query, key) pairs the mask
-leaves visible (causal: N(N+1)/2 pairs per slice), the work the kernel does,
-and the roofline fractions use that count.
+4*B*H*N^2*d per step over the step time (the metric as stated, causal runs
+included); `value_executed` counts only the (query, key) pairs the mask leaves
+visible (causal: N(N+1)/2 per slice), the work the kernel does, and the
+roofline fractions use that count.  With one GPU the line also carries:
+  per_config   every other point of the sweep (B4 H32, N 1K..32K, d 64/128,
+               causal and not) and the llm_prefill, video_dit and nvfp4
+               workloads, each timed the same way;
+  tensor_peaks the tensor-core rate probe (sage_probe_mma_rate) per
+               instruction kind, the denominators of the fractions;
+  accuracy     cos / relative L1 / RMSE of the output against fp64 attention
+               and max-abs against the CPU oracle, on sampled rows
+               (SageAttention2++ summary, App. A.2).
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -24,7 +33,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import signal
 import subprocess
@@ -40,24 +48,22 @@ sys.path.insert(0, ROOT)
 from quantized_attention_sub_b200 import api, inputs, replicas  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FP8_OVER_BF16 = 2.0   # nominal dense ratio 4.5 / 2.25 PFLOP/s (INT8 dense equals FP8 dense)
-# one metric for both arms: 4*B*H*N^2*d over the step time; the fraction of
-# the tensor peak is in `roofline`
+# nominal dense datasheet rates per GPU (TFLOP/s), context beside the probe
+NOMINAL_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0, "int8": 4500.0, "fp4": 9000.0}
 METRIC = "attention TOPS (4·B·H·N²·d/time) vs N; % of dense FP8/INT8 tensor peak"
-FP4_OVER_BF16 = 4.0   # nominal dense ratio 9 / 2.25 PFLOP/s
+HEADLINE = "sweep_N32768_d128_full"
 
-# DRAM bytes (read + write) of one attention launch at the workload's full
-# size, from one ncu capture of the kernel as it stands on a smaller case
-# (inputs still above L2), scaled by the token count (attention traffic is
-# the codes read once plus the output, linear in N).  null for other sizes.
-TRAFFIC_BYTES = {"llm_prefill": 129.9e6, "video_dit": 200.6e6, "nvfp4": 66.8e6}
+# DRAM bytes (read + write) of one attention launch of the headline workload:
+# one ncu capture of the kernel as it stands on B4 H32 N8192 d128 (inputs
+# above L2), scaled by the token count (non-causal attention traffic is the
+# codes read once plus the output, linear in N).  None until captured.
+TRAFFIC_BYTES = {}
 
-# per mode: tensor peak ratio to bf16, attention kernel, arithmetic description
+MODE_NAMES = ["INT8_FP8", "INT8_FP8_F16ACC", "NVFP4"]
 MODE_INFO = {
-    0: (FP8_OVER_BF16, "attn_i8f8_kernel", "int8 QK / e4m3 PV, fp32 softmax and accumulation"),
-    1: (FP8_OVER_BF16, "attn_i8f8_kernel (FP16 accumulator)",
-        "int8 QK / e4m3 PV, fp16 PV accumulation per 64 keys, fp32 softmax"),
-    2: (FP4_OVER_BF16, "attn_fp4_kernel", "e2m1 QK and PV with ue4m3 block scales, fp32 softmax and accumulation"),
+    0: ("attn_i8f8_kernel", "int8 QK / e4m3 PV, fp32 softmax and accumulation"),
+    1: ("attn_i8f8_kernel (FP16 accumulator)", "int8 QK / e4m3 PV, fp16 PV accumulation per 64 keys, fp32 softmax"),
+    2: ("attn_fp4_kernel", "e2m1 QK and PV with ue4m3 block scales, fp32 softmax and accumulation"),
 }
 
 
@@ -69,16 +75,13 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
-def dist_init():
-    return replicas.init("nccl")
-
-
-def barrier(ws):
-    replicas.barrier(ws)
-
-
-def allreduce_max(x, ws):
-    return replicas.max_over_ranks(x, ws, "cuda")
+def workload(name):
+    if name in inputs.WORKLOADS:
+        return inputs.WORKLOADS[name]
+    if name.startswith("sweep_"):
+        _, n, d, c = name.split("_")
+        return inputs.sweep(int(n[1:]), int(d[1:]), c == "causal")
+    raise SystemExit("unknown workload %s" % name)
 
 
 class ClockSampler:
@@ -127,12 +130,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def oracle_sample(w, max_rows):
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample(w, max_rows, threads=0):
     """The CPU oracle as it stands on a bounded sample of the workload: slice
     (b=0, h=0) quantized in full, attention for `max_rows` evenly spaced
-    query rows.  Returns (ops of the sampled rows at 4*d per key of the row,
-    all N keys, as the metric counts them; seconds; threads; rows)."""
+    query rows.  Returns (ops of the sampled rows at 4*d per key the row sees
+    -- all N keys, or i+1 for row i under a causal mask; seconds; threads;
+    rows)."""
     import oracle as orc
+    if threads:
+        orc.set_num_threads(threads)
     q, k, v = inputs.generate(inputs.variant(w, B=1, H=1))
     f = lambda t: t.float().reshape(1, w.N, w.d).numpy()
     rows = np.unique(np.linspace(0, w.N - 1, min(max_rows, w.N)).astype(np.int32))
@@ -144,8 +153,8 @@ def oracle_sample(w, max_rows):
         qz = orc.quantize_int8_fp8(f(q), f(k), f(v), smooth_q=w.smooth_q, mode=w.mode)
         orc.attention_int8_fp8(qz, w.causal, rows=rows)
     dt = time.perf_counter() - t0
-    ops = float(4.0 * w.d * w.N * len(rows))
-    return ops, dt, orc.num_threads(), len(rows)
+    keys = (rows.astype(np.float64) + 1.0).sum() if w.causal else float(w.N) * len(rows)
+    return float(4.0 * w.d * keys), dt, orc.num_threads(), len(rows)
 
 
 def run_reference(args, w, ws, rank):
@@ -162,142 +171,197 @@ def run_reference(args, w, ws, rank):
         tot_ops += ops
         tot_t += dt
     value = tot_ops / tot_t / 1e12
-    sample = "slice (b0,h0) of %s quantized in full + attention of %d evenly spaced query rows per step" % (w.name, nr)
+    sample = ("slice (b0,h0) of %s quantized in full + attention of %d evenly spaced query rows per step "
+              "(ops counted over the keys each row sees)" % (w.name, nr))
     line = {"impl": "reference", "metric": METRIC, "value": value,
             "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": MODE_INFO[w.mode][2] + " (CPU oracle)", "data": "synthetic",
-            "config": config_of(w, args, ws),
+            "vs_baseline": None, "dtype": MODE_INFO[w.mode][1] + " (CPU oracle)", "data": "synthetic",
+            "config": config_of(w, ws),
             "cpu_baseline": {"value": value, "unit": "TOPS", "cores": thr, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, args, ws):
+def config_of(w, ws):
     return {"workload": w.name, "B": w.B * ws, "H": w.H, "N": w.N, "d": w.d, "dtype": w.dtype,
-            "causal": w.causal, "mode": ["INT8_FP8", "INT8_FP8_F16ACC", "NVFP4"][w.mode], "smooth_q": w.smooth_q,
+            "causal": w.causal, "mode": MODE_NAMES[w.mode], "smooth_q": w.smooth_q,
             "parallelism": "replicas x%d (independent (b,h) slices per rank)" % ws,
             "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no flush" % (
                 w.B * w.H * w.N * w.d * 2 / 1e6)}
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llm_prefill")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--N", type=int, default=0,
-                    help="override the workload's sequence length (small cases for profiling; "
-                         "the headline runs use the workload's own N)")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
+# --------------------------------------------------------------------------
+# Tensor-core rate probe
+# --------------------------------------------------------------------------
+PROBE_KINDS = {"int8": api.PROBE_I8, "fp8_f32acc": api.PROBE_F8_F32ACC, "fp8_f16acc": api.PROBE_F8_F16ACC,
+               "bf16": api.PROBE_BF16, "fp4": api.PROBE_FP4}
 
-    w = inputs.WORKLOADS[args.workload] if args.workload in inputs.WORKLOADS else None
-    if w is None and args.workload.startswith("sweep_"):
-        _, n, d, c = args.workload.split("_")
-        w = inputs.sweep(int(n[1:]), int(d[1:]), c == "causal")
-    if args.N > 0:
-        w = inputs.variant(w, N=args.N)
-    ws, rank, local = dist_init() if args.impl == "ours" or int(os.environ.get("WORLD_SIZE", "1")) > 1 else (1, 0, 0)
 
-    if args.impl == "reference":
-        run_reference(args, w, ws, rank)
-        if ws > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
+def probe_peaks(dev, sm_count):
+    """TFLOP/s of back-to-back tcgen05.mma per kind, one CTA per SM: `burst`
+    = one ~20 ms launch after a warm-up launch (the rate a kernel timed alone
+    sees), `sustained` = back-to-back launches for ~1.5 s (under the power
+    cap).  Each figure is the CUDA-event time of its launches."""
+    wsb = api.alloc_workspace(1, 1, 128, 64, 0, dev)
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, kind in PROBE_KINDS.items():
+        ops1 = api.sage_probe_mma_rate(kind, sm_count, 256, wsb, wsb.numel(), stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        api.sage_probe_mma_rate(kind, sm_count, 256, wsb, wsb.numel(), stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_small = e0.elapsed_time(e1) * 1e-3
+        # size one launch at ~20 ms from the small one's rate
+        iters = int(min(1 << 20, max(256, 256 * 0.02 / max(t_small, 1e-6))))
+        time.sleep(0.2)
+        e0.record(stream)
+        ops = api.sage_probe_mma_rate(kind, sm_count, iters, wsb, wsb.numel(), stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        burst = ops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        n_launch = 75
+        e0.record(stream)
+        for _ in range(n_launch):
+            api.sage_probe_mma_rate(kind, sm_count, iters, wsb, wsb.numel(), stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sustained = n_launch * ops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        out[name] = {"burst": burst, "sustained": sustained, "unit": "TFLOP/s",
+                     "launch": "%d CTAs x %d x 4 MMAs M128 N256" % (sm_count, iters)}
+        del ops1
+    api.sage_check(wsb, wsb.numel(), stream)
+    out["fp8_f16acc_over_f32acc"] = out["fp8_f16acc"]["burst"] / out["fp8_f32acc"]["burst"]
+    return out
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+
+def mode_peak(mode, probe, which="burst"):
+    """Tensor peak of one attention step's mix: half the operations are the
+    QK^T product, half the PV product, so the peak is the harmonic mean of
+    the two instruction rates (INT8 and FP8 with the mode's accumulator), or
+    the FP4 rate."""
+    if mode == 2:
+        return probe["fp4"][which]
+    pv = probe["fp8_f16acc" if mode == 1 else "fp8_f32acc"][which]
+    return 2.0 / (1.0 / probe["int8"][which] + 1.0 / pv)
+
+
+# --------------------------------------------------------------------------
+# Device timing of one workload
+# --------------------------------------------------------------------------
+def time_workload(w, dev, steps, warmup, seed_rank=0, clocks=None, ws=1):
+    """Quantize + attention steps on device-resident inputs; CUDA events on
+    the launch stream around each kernel group.  Returns the timings and the
+    tensors (for the accuracy and e2e legs)."""
     B, H, N, d = w.shape()
     dcode = api.DTYPE_CODE[inputs.DTYPES[w.dtype]]
-    # each rank draws its own slice batch (seed offset by rank)
-    wr = inputs.variant(w, seed=replicas.rank_seed(w.seed, rank))
+    wr = inputs.variant(w, seed=replicas.rank_seed(w.seed, seed_rank))
     q, k, v = [t.to(dev) for t in inputs.generate(wr, device="cuda")]
     out = torch.empty_like(q)
     wsbuf = api.alloc_workspace(B, H, N, d, w.mode, dev)
     nbytes = wsbuf.numel()
     stream = torch.cuda.current_stream()
 
-    def step():
-        ev_q.record(stream)
+    def step(ev):
+        ev[0].record(stream)
         api.sage_quantize_qkv(q, k, v, dcode, B, H, N, d, w.smooth_q, w.mode, wsbuf, nbytes, stream)
-        ev_a.record(stream)
+        ev[1].record(stream)
         api.sage_attn_quantized(wsbuf, nbytes, out, dcode, B, H, N, d, w.causal, w.smooth_q, w.mode, stream)
-        ev_b.record(stream)
+        ev[2].record(stream)
 
-    ev_q, ev_a, ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    for _ in range(args.warmup):
-        step()
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+    for i in range(warmup):
+        step(evs[i % steps])
     api.sage_check(wsbuf, nbytes, stream)
-
-    # timed region: K steps; per-step attention-kernel events on the launch stream
-    attn_ms = []
-    ev_pairs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    barrier(ws)
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
+    replicas.barrier(ws)
     torch.cuda.synchronize()
     t_start.record(stream)
-    for i in range(args.steps):
-        ev_q, ev_a, ev_b = ev_pairs[i]
-        step()
+    for i in range(steps):
+        step(evs[i])
     t_stop.record(stream)
     torch.cuda.synchronize()
-    barrier(ws)
-    clk = clocks.stop()
+    replicas.barrier(ws)
+    clk = clocks.stop() if clocks is not None else None
     api.sage_check(wsbuf, nbytes, stream)
-    ms = t_start.elapsed_time(t_stop) / args.steps
-    attn_ms = [a_.elapsed_time(b_) for _, a_, b_ in ev_pairs]
-    quant_ms = [q_.elapsed_time(a_) for q_, a_, _ in ev_pairs]
-    ms = allreduce_max(ms, ws)
-    attn_avg = allreduce_max(float(np.mean(attn_ms)), ws)
-    quant_avg = allreduce_max(float(np.mean(quant_ms)), ws)
+    ms = t_start.elapsed_time(t_stop) / steps
+    attn_ms = float(np.mean([a.elapsed_time(b) for _, a, b in evs]))
+    quant_ms = float(np.mean([s.elapsed_time(a) for s, a, _ in evs]))
+    return dict(ms=ms, attn_ms=attn_ms, quant_ms=quant_ms, clocks=clk, q=q, k=k, v=v, out=out, ws=wsbuf,
+                dcode=dcode)
 
-    ops_visible = inputs.executed_ops(w) * ws
-    ops_square = inputs.attention_ops(w) * ws
-    value = replicas.job_throughput(inputs.attention_ops(w), ms, ws) / 1e12
 
-    # roofline of the dominant kernel (attention), live CUDA-event time
-    peaks, peak_src = load_peaks()
-    ratio, kname, dtype_desc = MODE_INFO[w.mode]
-    peak_fp8 = peaks["bf16_tflops_sustained"] * ratio
-    achieved = inputs.executed_ops(w) / (attn_avg * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak_fp8,
-                "unit": "TFLOP/s", "frac": achieved / peak_fp8,
-                "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense %s : BF16 ratio)" % (
-                    peak_src, ratio, "FP4" if w.mode == 2 else "FP8/INT8"),
-                "traffic": TRAFFIC_BYTES.get(w.name) if args.N == 0 else None,
-                "traffic_unit": "bytes per launch", "attn_ms": attn_avg}
-    # the quantization pass (HBM-bound): 16-bit Q, K, V read once, int8/e4m3
-    # codes written, statistics and scales (small) not counted
+def quant_bytes(w):
+    """Algorithmic bytes of the quantization pass: 16-bit Q, K, V read once,
+    the codes written once (INT8/e4m3: 1 byte; NVFP4: half a byte plus 1/16
+    byte of block scale); statistics and per-granule scales not counted."""
+    B, H, N, d = w.shape()
     Np = (N + 127) // 128 * 128
-    # NVFP4: half a byte of code plus 1/16 byte of block scale per element
-    q_bytes = 3 * B * H * N * d * 2 + (3 * B * H * Np * d * 9 // 16 if w.mode == 2 else 3 * B * H * Np * d)
-    hbm = peaks["hbm_gbs"]
-    quant_line = {"bound": "hbm", "kernel": "quant_pass_kernel (stats) + quant_fold_kernel + quant_pass_kernel (codes)", "ms": quant_avg,
-                  "algorithmic_bytes": q_bytes, "achieved": q_bytes / (quant_avg * 1e-3) / 1e9,
-                  "peak": hbm, "unit": "GB/s", "frac": q_bytes / (quant_avg * 1e-3) / 1e9 / hbm}
+    return 3 * B * H * N * d * 2 + (3 * B * H * Np * d * 9 // 16 if w.mode == 2 else 3 * B * H * Np * d)
 
-    # End to end through the C ABI with host buffers (pinned): every step's
-    # host->device copy of Q, K, V and device->host copy of O are inside the
-    # timed region.  Steps are pipelined the way a serving loop runs them:
-    # step i+1's inputs cross the host link while step i computes and step
-    # i-1's output comes back (two device buffer sets; copy-in, compute and
-    # copy-out on their own streams, ordered by events).
-    hq, hk, hv = [t.cpu().pin_memory() for t in (q, k, v)]
+
+def summarize(w, t, probe, hbm):
+    """Figures of one timed workload (single rank)."""
+    ex = inputs.executed_ops(w)
+    attn_tops = ex / (t["attn_ms"] * 1e-3) / 1e12
+    qb = quant_bytes(w)
+    s = {"workload": w.name, "mode": MODE_NAMES[w.mode], "causal": w.causal,
+         "ms_per_step": t["ms"], "value": inputs.attention_ops(w) / (t["ms"] * 1e-3) / 1e12,
+         "value_executed": ex / (t["ms"] * 1e-3) / 1e12,
+         "attn_ms": t["attn_ms"], "attn_tops_executed": attn_tops,
+         "quant_ms": t["quant_ms"], "quant_gbs": qb / (t["quant_ms"] * 1e-3) / 1e9,
+         "quant_frac_hbm": qb / (t["quant_ms"] * 1e-3) / 1e9 / hbm}
+    if probe is not None:
+        s["attn_frac_of_probe_burst"] = attn_tops / mode_peak(w.mode, probe)
+    return s
+
+
+def accuracy_leg(w, t, rows_n=48):
+    """cos / rel-L1 / RMSE of the GPU output against fp64 attention of the
+    unquantized inputs, and max-abs / rel-L1 against the CPU oracle, on
+    `rows_n` sampled query rows of slice (b0, h0)."""
+    import oracle as orc
+    B, H, N, d = w.shape()
+    f = lambda x: x.reshape(B * H, N, d)[:1].float().cpu().numpy()
+    q, k, v = f(t["q"]), f(t["k"]), f(t["v"])
+    rows = np.unique(np.linspace(0, N - 1, rows_n).astype(np.int32))
+    got = t["out"].reshape(B * H, N, d)[:1, rows].float().cpu().numpy()
+    ref64 = orc.attention_fp64(q, k, v, w.causal, rows=rows)
+    if w.mode == 2:
+        o32 = orc.attention_nvfp4(orc.quantize_nvfp4(q, k, v, smooth_q=w.smooth_q), w.causal, rows=rows)
+    else:
+        o32 = orc.attention_int8_fp8(orc.quantize_int8_fp8(q, k, v, smooth_q=w.smooth_q, mode=w.mode), w.causal,
+                                     rows=rows)
+    o_ref = torch.from_numpy(o32).to(inputs.DTYPES[w.dtype]).float().numpy()
+    diff = np.abs(got.astype(np.float64) - o_ref)
+    return {"vs_fp64": orc.accuracy(got, ref64), "vs_oracle": {
+        "max_abs": float(diff.max()), "rel_l1": float(diff.sum() / np.abs(o_ref).sum())},
+        "sample": "slice (b0,h0), %d evenly spaced query rows" % len(rows)}
+
+
+def e2e_leg(w, t, dev, steps, ws):
+    """End to end through the C ABI with host buffers (pinned): every step's
+    host->device copy of Q, K, V and device->host copy of O are inside the
+    timed region.  Steps are pipelined the way a serving loop runs them:
+    step i+1's inputs cross the host link while step i computes and step
+    i-1's output comes back (two device buffer sets; copy-in, compute and
+    copy-out on their own streams, ordered by events)."""
+    B, H, N, d = w.shape()
+    q, k, v, out, wsbuf = t["q"], t["k"], t["v"], t["out"], t["ws"]
+    nbytes = wsbuf.numel()
+    stream = torch.cuda.current_stream()
+    hq, hk, hv = [x.cpu().pin_memory() for x in (q, k, v)]
     houts = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    dins = [[torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)] for _ in range(2)]
-    douts = [torch.empty_like(out) for _ in range(2)]
+    dins = [[q, k, v], [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]]
+    douts = [out, torch.empty_like(out)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_run(nsteps):
+    def run(nsteps):
         ev_in = [torch.cuda.Event() for _ in range(nsteps)]
         ev_c = [torch.cuda.Event() for _ in range(nsteps)]
         ev_out = [torch.cuda.Event() for _ in range(nsteps)]
@@ -313,7 +377,7 @@ def main():
             if i >= 2:
                 stream.wait_event(ev_out[i - 2])  # this slot's output has been copied out
             api.sage_attn_fwd(dins[sl][0], dins[sl][1], dins[sl][2], douts[sl], B, H, N, d, w.causal, w.mode,
-                              dcode, w.smooth_q, wsbuf, nbytes, stream)
+                              t["dcode"], w.smooth_q, wsbuf, nbytes, stream)
             ev_c[i].record(stream)
             s_out.wait_event(ev_c[i])
             with torch.cuda.stream(s_out):
@@ -321,42 +385,153 @@ def main():
             ev_out[i].record(s_out)
         return ev_out[-1]
 
-    e2e_run(2)
+    run(2)
     torch.cuda.synchronize()
-    barrier(ws)
+    replicas.barrier(ws)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(4, min(args.steps, 12))
     e0.record(s_in)
-    last = e2e_run(e2e_steps)
+    last = run(steps)
     s_out.wait_event(last)
     e1.record(s_out)
     torch.cuda.synchronize()
-    e2e_ms = allreduce_max(e0.elapsed_time(e1) / e2e_steps, ws)
+    e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1) / steps, ws, "cuda")
     api.sage_check(wsbuf, nbytes, stream)
     in_bytes = 3 * q.numel() * q.element_size()
     out_bytes = out.numel() * out.element_size()
+    return {"value": inputs.attention_ops(w) * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
+            "pipelined": "step i+1's H2D copy overlaps step i's compute and step i-1's D2H copy"}
+
+
+def per_config_leg(dev, steps, probe, hbm, skip):
+    names = ["sweep_N%d_d%d_%s" % (n, d, c) for d in (128, 64) for c in ("full", "causal")
+             for n in (1024, 2048, 4096, 8192, 16384, 32768)]
+    names += ["llm_prefill", "video_dit", "nvfp4"]
+    res = {}
+    for name in names:
+        if name == skip:
+            continue
+        w = workload(name)
+        t = time_workload(w, dev, steps, 3)
+        res[name] = summarize(w, t, probe, hbm)
+        del t
+        torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the per-config sweep, the tensor-core probe and the accuracy leg")
+    ap.add_argument("--N", type=int, default=0,
+                    help="override the workload's sequence length (small cases for profiling; "
+                         "the headline runs use the workload's own N)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    w = workload(args.workload)
+    if args.N > 0:
+        w = inputs.variant(w, N=args.N)
+    ws, rank, local = replicas.init("nccl") if args.impl == "ours" or int(
+        os.environ.get("WORLD_SIZE", "1")) > 1 else (1, 0, 0)
+
+    if args.impl == "reference":
+        run_reference(args, w, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    peaks, peak_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    extras = ws == 1 and not args.no_extras
+
+    probe = probe_peaks(dev, sm_count) if extras else None
+
+    clocks = ClockSampler(local)
+    t = time_workload(w, dev, args.steps, args.warmup, seed_rank=rank, clocks=clocks, ws=ws)
+    ms = replicas.max_over_ranks(t["ms"], ws, "cuda")
+    attn_avg = replicas.max_over_ranks(t["attn_ms"], ws, "cuda")
+    quant_avg = replicas.max_over_ranks(t["quant_ms"], ws, "cuda")
+    value = replicas.job_throughput(inputs.attention_ops(w), ms, ws) / 1e12
+
+    # roofline of the dominant kernel (attention), live CUDA-event time
+    kname, dtype_desc = MODE_INFO[w.mode]
+    achieved = inputs.executed_ops(w) / (attn_avg * 1e-3) / 1e12
+    nominal = NOMINAL_TFLOPS["fp4" if w.mode == 2 else "fp8"]
+    if probe is not None:
+        peak = mode_peak(w.mode, probe, "burst")
+        peak_source = ("tensor-core probe (sage_probe_mma_rate), burst: harmonic mean of the INT8 and FP8 "
+                       "(accumulator of the mode) rates, half the operations each" if w.mode != 2 else
+                       "tensor-core probe (sage_probe_mma_rate), burst: block-scaled FP4 rate")
+    else:
+        peak = peaks["bf16_tflops"] * (4.0 if w.mode == 2 else 2.0)
+        peak_source = "%s bf16_tflops (burst) x nominal dense %s:BF16 ratio" % (peak_src, "FP4" if w.mode == 2
+                                                                              else "FP8")
+    traffic = TRAFFIC_BYTES.get(w.name) if args.N == 0 else None
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": peak_source,
+                "frac_of_nominal": achieved / nominal,
+                "nominal": "%.0f TFLOP/s dense datasheet" % nominal,
+                "traffic": traffic, "traffic_unit": "bytes per launch", "attn_ms": attn_avg,
+                "algorithmic_ops_per_launch": inputs.executed_ops(w)}
+    qb = quant_bytes(w)
+    quant_line = {"bound": "hbm", "kernel": "quant_pass_kernel (stats) + quant_fold_kernel + quant_pass_kernel (codes)",
+                  "ms": quant_avg, "algorithmic_bytes": qb, "achieved": qb / (quant_avg * 1e-3) / 1e9,
+                  "peak": hbm, "unit": "GB/s", "frac": qb / (quant_avg * 1e-3) / 1e9 / hbm,
+                  "peak_source": "%s hbm_gbs" % peak_src}
+
+    acc = accuracy_leg(w, t) if rank == 0 and extras else None
+    e2e = e2e_leg(w, t, dev, max(4, min(args.steps, 12)), ws)
+    clk = t["clocks"]
+    del t
+    torch.cuda.empty_cache()
+
+    per_config = per_config_leg(dev, min(args.steps, 10), probe, hbm, w.name) if extras else None
 
     line = {"metric": METRIC, "value": value,
             "unit": "TOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dtype_desc, "data": "synthetic",
-            "config": config_of(w, args, ws),
-            "value_executed": ops_visible / (ms * 1e-3) / 1e12,
+            "config": config_of(w, ws),
+            "value_executed": inputs.executed_ops(w) * ws / (ms * 1e-3) / 1e12,
             "roofline": roofline,
             "quant_roofline": quant_line,
-            "e2e": {"value": ops_square / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
-                    "pipelined": "step i+1's H2D copy overlaps step i's compute and step i-1's D2H copy"},
+            "e2e": e2e,
             # per step: the stats, fold and codes quantization kernels and the attention kernel
             "gpu_launches": 4 * args.steps,
             "clocks": clk}
+    if probe is not None:
+        line["tensor_peaks"] = probe
+    if acc is not None:
+        line["accuracy"] = acc
+    if per_config is not None:
+        line["per_config"] = per_config
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle as orc
         orc.build()
         ops, dt, thr, nr = oracle_sample(w, 2048)
-        line["cpu_baseline"] = {"value": ops / dt / 1e12, "unit": "TOPS", "cores": thr, "kind": "oracle",
-                                "sample": "slice (b0,h0) quantized in full + attention of %d evenly spaced "
-                                          "query rows; %.1f s" % (nr, dt)}
+        cpu = {"value": ops / dt / 1e12, "unit": "TOPS", "cores": thr, "kind": "oracle",
+               "sample": "slice (b0,h0) quantized in full + attention of %d evenly spaced query rows; %.1f s "
+                         "(ops counted over the keys each row sees)" % (nr, dt)}
+        if extras:
+            single = {}
+            for name, rows_n in (("unit", 128), ("llm_prefill", 64)):
+                o1, d1, _, n1 = oracle_sample(workload(name), rows_n, threads=1)
+                single[name] = {"value": o1 / d1 / 1e12, "unit": "TOPS", "seconds": d1, "rows": n1}
+            orc.set_num_threads(thr)
+            cpu["single_thread"] = single
+        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

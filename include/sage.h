@@ -188,6 +188,21 @@ SAGE_API sage_status sage_debug_fp4_s(const void* ws, size_t ws_bytes, int B, in
  * error word at offset 0 of `ws` (>= 4 bytes, 1024-byte aligned). */
 SAGE_API sage_status sage_debug_timeout_probe(void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* Tensor-core rate probe, the denominator of the library's roofline
+ * fractions (the pages measure instruction speedups in the SageAttention2++
+ * summary, Sec. 2.2, Table 1: FP8 with an FP16 accumulator against FP8 with
+ * an FP32 one).  Launches `ctas` CTAs (one per SM: each allocates 512 TMEM
+ * columns) that each issue `iters` x 4 back-to-back tcgen05.mma of one kind,
+ * M = 128, N = 256, on operand tiles resident in shared memory, and returns
+ * in *ops (may be NULL) the operation count 2*M*N*K summed over all of them.
+ * The caller times the launch (events on `stream`) and divides.  kind: one of
+ * the SAGE_PROBE_* values.  iters <= 2^20; keep one launch under a second
+ * (the completion wait is bounded at 2 s and reports SAGE_ERR_TIMEOUT through
+ * sage_check).  Uses only the error word at offset 0 of `ws`. */
+enum { SAGE_PROBE_I8 = 0, SAGE_PROBE_F8_F32ACC = 1, SAGE_PROBE_F8_F16ACC = 2, SAGE_PROBE_BF16 = 3, SAGE_PROBE_FP4 = 4 };
+SAGE_API sage_status sage_probe_mma_rate(int kind, int ctas, int iters, void* ws, size_t ws_bytes, double* ops,
+                                         sage_stream_t stream);
+
 /* Synchronize `stream`, then read and clear the workspace error word.
  * Returns SAGE_ERR_TIMEOUT if a kernel gave up a wait, SAGE_ERR_CUDA on a
  * CUDA error, else SAGE_OK. */

@@ -59,6 +59,17 @@ ORC_EXPORT int orc_num_threads(void)
 #endif
 }
 
+/* Set the number of host threads of the parallel loops (1: single-threaded
+ * timing). */
+ORC_EXPORT void orc_set_num_threads(int n)
+{
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------ */
 /* Small-float formats.                                                      */
 /* ------------------------------------------------------------------------ */

@@ -21,7 +21,9 @@ DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
 
 EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_quantize_qkv_static",
             "sage_attn_quantized",
-            "sage_attn_fwd", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_check", "sage_last_error")
+            "sage_attn_fwd", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_probe_mma_rate",
+            "sage_check", "sage_last_error")
+PROBE_I8, PROBE_F8_F32ACC, PROBE_F8_F16ACC, PROBE_BF16, PROBE_FP4 = range(5)
 
 
 class WsLayout(ctypes.Structure):
@@ -66,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.sage_debug_fp4_s.restype = i
         L.sage_debug_timeout_probe.argtypes = [vp, sz, vp]
         L.sage_debug_timeout_probe.restype = i
+        L.sage_probe_mma_rate.argtypes = [i, i, i, vp, sz, ctypes.POINTER(ctypes.c_double), vp]
+        L.sage_probe_mma_rate.restype = i
         L.sage_check.argtypes = [vp, sz, vp]
         L.sage_check.restype = i
         L.sage_last_error.argtypes = []
@@ -132,6 +136,14 @@ def sage_debug_fp4_s(ws, ws_bytes, B, H, N, d, bh, q_tile, k_tile, out, stream=N
 
 def sage_debug_timeout_probe(ws, ws_bytes, stream=None):
     _raise(lib().sage_debug_timeout_probe(_ptr(ws), ws_bytes, _stream(stream)))
+
+
+def sage_probe_mma_rate(kind, ctas, iters, ws, ws_bytes, stream=None) -> float:
+    """Launch the tensor-core rate probe; returns the operation count of the
+    launch (the caller times it with events on the same stream)."""
+    ops = ctypes.c_double(0.0)
+    _raise(lib().sage_probe_mma_rate(kind, ctas, iters, _ptr(ws), ws_bytes, ctypes.byref(ops), _stream(stream)))
+    return ops.value
 
 
 def sage_check(ws, ws_bytes, stream=None):

@@ -299,6 +299,19 @@ sage_status sage_debug_timeout_probe(void* ws, size_t ws_bytes, sage_stream_t st
   return cuda_status(sage::launch_timeout_probe(resolve(ws, L), (cudaStream_t)stream), "probe launch");
 }
 
+sage_status sage_probe_mma_rate(int kind, int ctas, int iters, void* ws, size_t ws_bytes, double* ops,
+                               sage_stream_t stream) {
+  if (!ws || ws_bytes < sizeof(int) || ((uintptr_t)ws) % kAlign)
+    return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null or misaligned%s");
+  if (kind < SAGE_PROBE_I8 || kind > SAGE_PROBE_FP4) return set_err(SAGE_ERR_INVALID_ARG, "unknown probe kind%s");
+  if (ctas < 1 || ctas > 65535 || iters < 1 || iters > (1 << 20))
+    return set_err(SAGE_ERR_INVALID_ARG, "ctas must be in [1, 65535] and iters in [1, 2^20]%s");
+  if (ops) *ops = sage::mma_rate_ops(kind, ctas, iters);
+  sage_status st = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream), "clear");
+  if (st != SAGE_OK) return st;
+  return cuda_status(sage::launch_mma_rate(kind, ctas, iters, (int*)ws, (cudaStream_t)stream), "probe launch");
+}
+
 sage_status sage_check(void* ws, size_t ws_bytes, sage_stream_t stream) {
   if (!ws || ws_bytes < sizeof(int)) return set_err(SAGE_ERR_INVALID_ARG, "workspace pointer is null%s");
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

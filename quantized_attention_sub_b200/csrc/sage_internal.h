@@ -91,6 +91,12 @@ cudaError_t launch_debug_qk(const WsPtrs& w, const Problem& pb, int bh, int q_ti
 cudaError_t launch_debug_fp4_s(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, float* out,
                                cudaStream_t s);
 
+// Tensor-core rate probe (probe.cu): `ctas` CTAs each issue `iters` x 4
+// back-to-back M=128 N=256 MMAs of one kind on shared-memory operands.
+enum { kProbeI8 = 0, kProbeF8F32 = 1, kProbeF8F16 = 2, kProbeBF16 = 3, kProbeFP4 = 4 };
+cudaError_t launch_mma_rate(int kind, int ctas, int iters, int* err, cudaStream_t s);
+double mma_rate_ops(int kind, int ctas, int iters);  // 2*M*N*K per instruction, summed
+
 // A kernel whose only wait can never complete: exercises the bounded-wait path.
 cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s);
 

@@ -17,7 +17,9 @@ reasons, and counted:
             oracle's own figure for the element: the largest change that one
             P~ code (NVFP4: one P~ block) moved by one step would cause,
             step(P~_j) * |v_jc| * scale_v / (Pr * l) over the row's keys.
-            At most 1e-3 of the elements (at least 4) may use it.
+            A moved code shifts its whole output row, so the count is of
+            rows: at most 2 % of the compared rows (at least 2) may hold such
+            elements.
 
 The relative L1 bound covers every element.
 """
@@ -25,7 +27,7 @@ import numpy as np
 import torch
 
 MAX_ABS, REL_L1 = 2e-3, 5e-4
-P_CODE_SHARE = 1e-3
+P_CODE_ROW_SHARE = 0.02
 
 DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
 
@@ -60,14 +62,18 @@ def compare_out(o_gpu, ref32, flip, dtype, label=""):
     p_bound = MAX_ABS + np.asarray(flip, np.float64) + _half_ulp(o_gpu, dtype)
     p_code = rest & (np.abs(a - y) <= p_bound)
     bad = rest & ~p_code
-    n_p_allowed = max(4, int(P_CODE_SHARE * diff.size))
+    rows = p_code.reshape(-1, p_code.shape[-1]).any(axis=1) if p_code.ndim else p_code
+    n_rows = max(1, rows.size)
+    n_p_allowed = max(2, int(np.ceil(P_CODE_ROW_SHARE * n_rows)))
     rel = float(diff.sum() / max(np.abs(ref).sum(), 1e-30))
-    stats = dict(label=str(label), elements=int(diff.size), max_abs=float(diff.max()) if diff.size else 0.0,
+    stats = dict(label=str(label), elements=int(diff.size), rows=int(n_rows),
+                 max_abs=float(diff.max()) if diff.size else 0.0,
                  rel_l1=rel, over_2e3=int(over.sum()), boundary=int(boundary.sum()), p_code=int(p_code.sum()),
+                 p_code_rows=int(rows.sum()),
                  p_code_max_abs=float(diff[p_code].max()) if p_code.any() else 0.0,
                  max_abs_plain=float(np.where(over, 0.0, diff).max()) if diff.size else 0.0)
     print("parity", stats)
-    assert int(bad.sum()) == 0 and int(p_code.sum()) <= n_p_allowed and rel <= REL_L1, (
+    assert int(bad.sum()) == 0 and int(rows.sum()) <= n_p_allowed and rel <= REL_L1, (
         stats, "unexplained" if bad.any() else "", np.argwhere(bad)[:5].tolist(),
         float(diff[bad].max()) if bad.any() else 0.0)
     return stats
