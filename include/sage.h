@@ -163,6 +163,20 @@ SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, 
                           int causal, int mode, int dtype, int smooth_q, void* ws, size_t ws_bytes,
                           sage_stream_t stream);
 
+/* sage_attn_fwd with the P~ and V quantization ranges chosen by the caller:
+ * P~ = e4m3(p * Pr), V codes e4m3(v * Vr / absmax), O rescaled by 1 / Pr.
+ * The SageAttention2++ summary (Sec. 3.1) narrows both so that an FP16
+ * accumulator cannot overflow and picks Pr = 224, Vr = 4.5 among the pairs
+ * that qualify; sage_attn_fwd uses those (448, 448 with the FP32
+ * accumulator).  Pr and Vr must lie in (0, 448]; in
+ * SAGE_MODE_INT8_FP8_F16ACC the worst 64-key FP16 partial, 64 * Pr * Vr,
+ * must not exceed 65504 -- otherwise SAGE_ERR_INVALID_ARG.  SAGE_MODE_NVFP4
+ * returns SAGE_ERR_UNSUPPORTED (its P~ scale is fixed).  Other arguments as
+ * for sage_attn_fwd. */
+SAGE_API sage_status sage_attn_fwd_ranges(const void* q, const void* k, const void* v, void* out, int B, int H,
+                                          int N, int d, int causal, int mode, int dtype, int smooth_q, float Pr,
+                                          float Vr, void* ws, size_t ws_bytes, sage_stream_t stream);
+
 /* Parity helper: the INT32 tile S = Q^ K^T of query tile `q_tile` and key tile
  * `k_tile` (128 x 128) of slice `bh`, computed by the same tensor-core path as
  * the attention kernel (kind::i8 MMA, accumulator in TMEM).  out: device

@@ -143,6 +143,27 @@ bool make_tmap_u8_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t d
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8_nd(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                     const uint32_t* box, int swizzle_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace sage
 
 extern "C" {
@@ -162,8 +183,25 @@ size_t sage_workspace_size(int B, int H, int N, int d, int mode) {
   return layout_of(B, H, N, d, mode).total;
 }
 
+// Default quantization ranges of a mode (SageAttention2++ summary, Sec. 3.1:
+// Pr = 224 and Vr = 4.5 with the FP16 accumulator; the full e4m3 range 448
+// with the FP32 one).
+static float default_vr(int mode) { return mode == SAGE_MODE_INT8_FP8_F16ACC ? 4.5f : 448.0f; }
+static float default_pr(int mode) { return mode == SAGE_MODE_INT8_FP8_F16ACC ? 224.0f : 448.0f; }
+
+static sage_status quantize(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
+                            int smooth_q, int mode, float Vr, void* ws, size_t ws_bytes, sage_stream_t stream);
+static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
+                                  int causal, int smooth_q, int mode, float Pr, sage_stream_t stream,
+                                  bool after_quantize);
+
 sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
                               int smooth_q, int mode, void* ws, size_t ws_bytes, sage_stream_t stream) {
+  return quantize(q, k, v, dtype, B, H, N, d, smooth_q, mode, default_vr(mode), ws, ws_bytes, stream);
+}
+
+static sage_status quantize(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
+                            int smooth_q, int mode, float Vr, void* ws, size_t ws_bytes, sage_stream_t stream) {
   sage_status st = check_shape(B, H, N, d, mode);
   if (st != SAGE_OK) return st;
   if (!q || !k || !v) return set_err(SAGE_ERR_INVALID_ARG, "null input pointer%s");
@@ -173,7 +211,6 @@ sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int d
   const sage_ws_layout L = layout_of(B, H, N, d, mode);
   if ((st = check_ws(ws, ws_bytes, L.total)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, 0};
-  const float Vr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 4.5f : 448.0f;
   if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
   return cuda_status(sage::launch_quant_int8_fp8(q, k, v, pb, Vr, resolve(ws, L), (cudaStream_t)stream),
@@ -204,7 +241,7 @@ sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v
     return SAGE_ERR_UNSUPPORTED;
   }
   sage::Problem pb{B * H, N, (int)Np, d, dtype, smooth_q ? 1 : 0, mode, 0};
-  const float Vr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 4.5f : 448.0f;
+  const float Vr = default_vr(mode);
   if ((st = cuda_status(cudaMemsetAsync((char*)out + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
   return cuda_status(sage::launch_quant_static(q, k, v, pb, Vr, resolve(out, L), (cudaStream_t)stream),
@@ -215,7 +252,8 @@ sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v
 // sage_quantize_qkv on the same stream (sage_attn_fwd) the workspace error
 // word is already clear; called on its own it clears it first.
 static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
-                                  int causal, int smooth_q, int mode, sage_stream_t stream, bool after_quantize) {
+                                  int causal, int smooth_q, int mode, float Pr, sage_stream_t stream,
+                                  bool after_quantize) {
   sage_status st = check_shape(B, H, N, d, mode);
   if (st != SAGE_OK) return st;
   if (!out) return set_err(SAGE_ERR_INVALID_ARG, "null output pointer%s");
@@ -233,9 +271,6 @@ static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, in
     return cuda_status(
         sage::launch_attn_fp4(resolve(const_cast<void*>(ws), L), out, pb, (cudaStream_t)stream),
         "attention launch");
-  // Pr: full e4m3 range with the FP32 accumulator, 224 with the FP16 one
-  // (SageAttention2++ summary, Sec. 3.1)
-  const float Pr = mode == SAGE_MODE_INT8_FP8_F16ACC ? 224.0f : 448.0f;
   return cuda_status(
       sage::launch_attn_i8f8(resolve(const_cast<void*>(ws), L), out, pb, Pr, (cudaStream_t)stream),
       "attention launch");
@@ -243,7 +278,8 @@ static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, in
 
 sage_status sage_attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
                                 int causal, int smooth_q, int mode, sage_stream_t stream) {
-  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream, false);
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, default_pr(mode), stream,
+                        false);
 }
 
 sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
@@ -251,7 +287,25 @@ sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out
                           sage_stream_t stream) {
   sage_status st = sage_quantize_qkv(q, k, v, dtype, B, H, N, d, smooth_q, mode, ws, ws_bytes, stream);
   if (st != SAGE_OK) return st;
-  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, stream, true);
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, default_pr(mode), stream,
+                        true);
+}
+
+sage_status sage_attn_fwd_ranges(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                                 int causal, int mode, int dtype, int smooth_q, float Pr, float Vr, void* ws,
+                                 size_t ws_bytes, sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (mode == SAGE_MODE_NVFP4)
+    return set_err(SAGE_ERR_UNSUPPORTED, "the NVFP4 mode has no P~ / V ranges (its block scales are fixed)%s");
+  if (!(Pr > 0.0f && Pr <= 448.0f) || !(Vr > 0.0f && Vr <= 448.0f))
+    return set_err(SAGE_ERR_INVALID_ARG, "Pr and Vr must lie in (0, 448], the finite e4m3 range%s");
+  // the worst 64-key FP16 partial (all P~ = Pr, all |v^| = Vr) must stay finite
+  if (mode == SAGE_MODE_INT8_FP8_F16ACC && 64.0 * (double)Pr * (double)Vr > 65504.0)
+    return set_err(SAGE_ERR_INVALID_ARG, "64 * Pr * Vr exceeds 65504: the FP16 partial could overflow%s");
+  st = quantize(q, k, v, dtype, B, H, N, d, smooth_q, mode, Vr, ws, ws_bytes, stream);
+  if (st != SAGE_OK) return st;
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, Pr, stream, true);
 }
 
 sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,

@@ -8,19 +8,24 @@
 // One CTA owns two 128-query tiles of one (b, h) slice and walks the key
 // tiles of 128 in order (causal: the longest query blocks launch first, see
 // the grid mapping in the kernel).  Warp roles (576 threads, 18 warps):
-//   warps 0-15  softmax: warpgroup g = warp / 4 handles query tile q = g / 2
-//               and key half h = g % 2 (keys [64h, 64h + 64) of every tile,
-//               one 64-key scale granule); thread <-> row <-> TMEM lane.
-//               Each SM sub-partition runs one warp of every warpgroup.
+//   warps 0-15  softmax: warps 8q..8q+7 handle query tile q; warp w reads the
+//               16 TMEM lanes 32 (w%4) + 16 ((w/4)%2) .. +15 with the .16x64b
+//               shape, so the two threads of a row (lanes t and t^2) sit in one
+//               warp, one per 64-key half (one 64-key scale granule each).
 //   warp 16     TMA producer (Q tiles once, then a 3-stage ring of K and V^T
 //               tiles); owns the TMEM allocation
 //   warp 17     MMA issuer (one thread): S_q = Q_q K^T with tcgen05 kind::i8
 //               into TMEM, O_q += P~_q V with kind::f8f6f4 into TMEM
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 after it.
+// The K tile rows and the V^T tile rows (channels) arrive in shared memory in
+// pair order -- row 2i + e holds key (channel) 64e + i (d/2 e + i) -- through
+// the tensor maps' strides, so that in TMEM column 2i + e of S and O belongs
+// to half e: a .16x64b load hands each thread of a row one contiguous half of
+// the keys and of the output channels.
 // Per key tile j the two threads of row i (one per key half):
-//   load their 64 S values from TMEM and free the S buffer,
-//   take the half's logit max and exchange it through shared memory,
-//   m_new = max(m, both halves' max), alpha = exp2(m - m_new),
+//   load their 64 S values from TMEM and free the buffer,
+//   take the half's logit max and the row max with one shuffle,
+//   m_new = max(m, row max), alpha = exp2(m - m_new),
 //   p' = 2^d with d = t - m_new + log2(Pr), P~ = e4m3(p'),
 //   wait for the previous P~V, multiply their half of the O row by alpha
 //   (skipped when alpha == 1 on the whole warp), write their 64 P~ bytes into
@@ -28,9 +33,10 @@
 // At the end l = l_0 + l_1 and O = acc * scale_v / l is cast and stored (the
 // quotient through one reciprocal of l per row and an FMA correction).
 // exp2 runs on the special-function unit (ex2.approx; in the FP16 mode a
-// quarter on a polynomial, ex2_poly2); the CPU reference computation uses the
-// library exp2, so a P~ code may differ in rare cases and the output is
-// compared within a tolerance.
+// quarter on a polynomial, ex2_poly2); the logit is formed as
+// fma(x, (sq sk) log2(e)/sqrt(d), ...) and Pr enters the exponent, so a P~ code
+// may differ from the CPU reference's e4m3(p * Pr) in rare cases and the
+// output is compared within a tolerance.
 // Every wait is bounded (sage_ptx.cuh); a timeout records an error code in
 // the workspace, makes the other roles stop, and the CTA frees its TMEM.
 #include <cuda_bf16.h>
@@ -52,7 +58,7 @@ constexpr int kStages = 3;
 template <bool F16ACC>
 struct Roles {
   static constexpr int kNQ = F16ACC ? 1 : 2;
-  static constexpr int kSoftmaxWarps = 8 * kNQ;  // two key halves x 4 warps per query tile
+  static constexpr int kSoftmaxWarps = 8 * kNQ;  // 8 warps x 16 rows x 2 halves per query tile
   static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
 };
@@ -61,18 +67,15 @@ constexpr uint32_t kTmemCols = 512;
 template <int D, int NQ>
 struct Smem {
   static constexpr int kQ = 128 * D;  // one Q tile (int8)
-  static constexpr int kK = 128 * D;  // one K tile (int8)
-  static constexpr int kV = D * 128;  // one V^T tile (e4m3)
+  static constexpr int kK = 128 * D;  // one K tile (int8), rows in pair order
+  static constexpr int kV = D * 128;  // one V^T tile (e4m3), rows in pair order
   static constexpr int kP = 128 * 128;
   static constexpr int off_q = 0;
   static constexpr int off_k = off_q + NQ * kQ;
   static constexpr int off_v = off_k + kStages * kK;
   static constexpr int off_p = off_v + kStages * kV;  // [query tile NQ][buffer 2]
   static constexpr int off_bar = off_p + 2 * NQ * kP;
-  // row-max / row-sum exchange between the two key halves:
-  // [query tile 2][tile parity 2][half 2][row 128] floats
-  static constexpr int off_x = off_bar + 256;
-  static constexpr int bytes = off_x + 2 * 2 * 2 * 128 * 4;
+  static constexpr int bytes = off_bar + 256;
   static constexpr int alloc = bytes + 1024;  // room to align the base to 1024
 };
 
@@ -97,6 +100,7 @@ enum : int {
   kErrProbe = 0x1FF
 };
 
+SAGE_DEV float lo_half_to_float(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu))); }
 
 }  // namespace
 
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   // TMEM columns: S_q, O_q, and (FP16 accumulator) the two 64-key chunk partials H_c
   constexpr uint32_t kColO = F16ACC ? 128u : 256u;
   constexpr uint32_t kColH = 128u + D;
-  constexpr int kHalfD = D / 2;  // O columns each key half rescales and stores
+  constexpr int kHalfD = D / 2;  // O columns (channels) each thread of a row rescales and stores
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(smem + L::off_bar);
@@ -124,11 +128,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   uint64_t* s_free = s_full + 2;              // [2]
   uint64_t* p_full = s_full + 4;              // [2]
   uint64_t* o_done = s_full + 6;              // [2]
-  uint64_t* x_bar = s_full + 8;               // [2 query tiles][2 parities]
-  uint64_t* mma_fin = s_full + 12;
-  uint32_t* tmem_slot = (uint32_t*)(s_full + 13);
+  uint64_t* mma_fin = s_full + 8;
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 9);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* xch = (float*)(smem + L::off_x);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Grid (query blocks, B*H): one slice's CTAs launch together and share its
@@ -162,8 +164,6 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       mbar_init(&s_free[q], 8);   // 8 softmax warps per query tile
       mbar_init(&p_full[q], 8);
       mbar_init(&o_done[q], 1);
-      mbar_init(&x_bar[2 * q], 256);
-      mbar_init(&x_bar[2 * q + 1], 256);
     }
     mbar_init(mma_fin, 1);
     *abort_flag = 0;
@@ -197,14 +197,14 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(&k_full[s], L::kK);
-        tma_load_3d(smem + L::off_k + s * L::kK, &tm_k, &k_full[s], 0, j * 128, bh);
+        tma_load_5d(smem + L::off_k + s * L::kK, &tm_k, &k_full[s], 0, 0, 0, j, bh);
         issued_k = j + 1;
         if (j >= kStages && !mbar_wait(&v_empty[s], (n - 1) & 1, abort_flag)) {
           fail(abort_flag, a.err, kErrProducer);
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kV);
-        tma_load_3d(smem + L::off_v + s * L::kV, &tm_v, &v_full[s], j * 128, 0, bh);
+        tma_load_4d(smem + L::off_v + s * L::kV, &tm_v, &v_full[s], j * 128, 0, 0, bh);
         issued_v = j + 1;
       }
       // Drain: every load issued into shared memory must land before exit.
@@ -291,46 +291,48 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
     }
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
-    const int g = warp >> 2;          // warpgroup
-    const int q = g >> 1, h = g & 1;  // query tile, key half
-    const int r = threadIdx.x & 127;
-    const int w4 = warp & 3;
+    const int q = warp >> 3;                // query tile
+    const int wq = warp & 7;
+    const int h = (lane >> 1) & 1;          // key half and channel half of this thread
+    const int r = 32 * (wq & 3) + 16 * (wq >> 2) + (lane >> 2) + 8 * (lane & 1);
+    const uint32_t lane_off = (uint32_t)(32 * (wq & 3) + 16 * (wq >> 2)) << 16;
     if (nt[q] > 0) {
       const int qt = kNQ * qb + q;
       const int row = qt * 128 + r;
       const float sq = a.q_scale[(size_t)bh * (a.Npad / 32) + (row >> 5)];
-      const uint32_t lane_off = (uint32_t)(w4 * 32) << 16;
-      const uint32_t t_s = tmem + lane_off + q * 128 + h * 64;
-      const uint32_t t_o = tmem + lane_off + kColO + q * D + h * kHalfD;
-      const uint32_t t_h = tmem + lane_off + kColH + h * kHalfD;  // H_0 here, H_1 is D columns further
+      // S columns [0, 128) of this query tile (two loads of 64), O columns of this
+      // tile, H_0 (H_1 is D columns further)
+      const uint32_t t_s = tmem + lane_off + q * 128;
+      const uint32_t t_o = tmem + lane_off + kColO + q * D;
+      const uint32_t t_h = tmem + lane_off + kColH;
       uint8_t* prow0 = smem + L::off_p + 2 * q * L::kP + r * 128;  // buffer 0; buffer 1 is kP further
       const float* ksc = a.k_scale + (size_t)bh * (a.Npad / 64);
       const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
-      float* xq = xch + q * 512;  // [parity][half][row]
       // m: running row max of the logits (log2 units); l: this half's running
       // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
       float alpha_prev = 0.f;  // FP16 accumulator: rescale factor of the tile whose partials are pending
       bool ok = true;
       // FP16 accumulator, after P~V(jt) completed: acc = (alpha_jt * acc + h_0) + h_1
-      // over this half's O columns (the first tile starts from acc = 0).
+      // over this thread's O columns (the first tile starts from acc = 0).
       auto fold_partials = [&](int jt, float alpha_t) {
 #pragma unroll 1
-        for (int i = 0; i < kHalfD / 32; ++i) {
-          uint32_t o[32], h0[16], h1[16];
-          tmem_ld16_pack16(t_h + 32 * i, h0);
-          tmem_ld16_pack16(t_h + D + 32 * i, h1);
-          if (jt > 0) tmem_ld32(t_o + 32 * i, o);
+        for (int i = 0; i < D / 32; ++i) {
+          uint32_t o[16], h0[16], h1[16];
+          tmem_ld16x64b_x16(t_h + 32 * i, h0);
+          tmem_ld16x64b_x16(t_h + D + 32 * i, h1);
+          if (jt > 0) tmem_ld16x64b_x16(t_o + 32 * i, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float2 acc = jt > 0 ? __fmul2_rn(make_float2(u2f(o[2 * e]), u2f(o[2 * e + 1])), make_float2(alpha_t, alpha_t))
+          for (int e = 0; e < 16; e += 2) {
+            float2 acc = jt > 0 ? __fmul2_rn(make_float2(u2f(o[e]), u2f(o[e + 1])), make_float2(alpha_t, alpha_t))
                                 : make_float2(0.f, 0.f);
-            acc = __fadd2_rn(__fadd2_rn(acc, h2f2(h0[e])), h2f2(h1[e]));
-            o[2 * e] = f2u(acc.x);
-            o[2 * e + 1] = f2u(acc.y);
+            acc = __fadd2_rn(__fadd2_rn(acc, make_float2(lo_half_to_float(h0[e]), lo_half_to_float(h0[e + 1]))),
+                             make_float2(lo_half_to_float(h1[e]), lo_half_to_float(h1[e + 1])));
+            o[e] = f2u(acc.x);
+            o[e + 1] = f2u(acc.y);
           }
-          tmem_st32(t_o + 32 * i, o);
+          tmem_st16x64b_x16(t_o + 32 * i, o);
         }
         tmem_st_wait();
       };
@@ -347,9 +349,8 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           if (a.causal) lim = min(lim, row - kbase + 1);
         }
         // FP16 mode: the tile's 64 bias values, loaded before the wait for S
-        // hides their latency (measured faster than loading half of them ahead,
-        // despite a few spilled registers); the FP32 mode, whose 576 threads
-        // leave no registers for it, loads them where they are used
+        // hides their latency; the FP32 mode, whose 576 threads leave no
+        // registers for it, loads them where they are used
         constexpr int kAhead = F16ACC ? 16 : 0;
         float4 bv[HAS_BIAS && kAhead > 0 ? kAhead : 1];
         if (HAS_BIAS) {
@@ -363,18 +364,20 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           break;
         }
         tc_fence_after();
+        // sr[c] = S of key 64 h + c (int32, then as float)
         uint32_t sr[64];
-        tmem_ld32(t_s, sr);
-        tmem_ld32(t_s + 32, sr + 32);
+        tmem_ld16x64b_x32(t_s, sr);
+        tmem_ld16x64b_x32(t_s + 64, sr + 32);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[q]);
 
-        // Logits and P~ take the fp32 steps of the CPU reference computation:
+        // Logits:
         //   kf = (sq * sk) * log2(e)/sqrt(d) for this half's 64-key granule,
-        //   t  = float(S) * kf  (or fma(float(S), kf, bias * log2(e)/sqrt(d))),
-        //   m' = max - log2(Pr),  d = fma(float(S), kf, -m')  (or t - m'),
+        //   x  = float(S) (exact: |S| <= 128 * 127^2 < 2^24),
+        //   t  = x * kf  (or fma(x, kf, bias * log2(e)/sqrt(d))),
+        //   m' = max - log2(Pr),  d = fma(x, kf, -m')  (or t - m'),
         //   p' = 2^d = p * Pr on the special-function unit, P~ = e4m3(p').
         // Masked keys become -inf: out of the max, and 2^-inf = +0.  (A zero
         // scale -- an all-zero granule -- is raised to the smallest normal
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
             ga = fmax3(ga, u2f(sr[c]), u2f(sr[c + 1]));
             gb = fmax3(gb, u2f(sr[c + 2]), u2f(sr[c + 3]));
           }
-          // a half with no visible key gives -inf, or NaN for a zero scale
+          // a half with no visible key gives -inf
           mt = __fmul_rn(fmaxf(ga, gb), kf);
         } else {
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
@@ -413,21 +416,14 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
             sr[c + 1] = f2u(ta.y);
             sr[c + 2] = f2u(tb.x);
             sr[c + 3] = f2u(tb.y);
-            // masked keys carry -inf (or NaN for a zero scale): fmax3 ignores NaN
+            // masked keys carry -inf
             ma = fmax3(ma, ta.x, ta.y);
             mb = fmax3(mb, tb.x, tb.y);
           }
           mt = fmaxf(ma, mb);
         }
-        // exchange the half maxima of the row (slot parity alternates per tile)
-        float* xs = xq + (j & 1) * 256;
-        xs[h * 128 + r] = mt;
-        mbar_arrive(&x_bar[2 * q + (j & 1)]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&x_bar[2 * q + (j & 1)], (j >> 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        mt = fmaxf(mt, xs[(h ^ 1) * 128 + r]);
+        // the row max: the other half of the row is lane ^ 2 of this warp
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
         const float m_new = fmaxf(m, mt);
         const float alpha = ex2(__fadd_rn(m, -m_new));  // +0 on the first tile (m = -inf), 1 if the max stays
         const float mp = __fadd_rn(m_new, -a.log2Pr);
@@ -445,10 +441,10 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 16 * cc + 4 * e;
-            // d = t - m' (one rounding: fma(x, kf, -m') without bias)
-            const float2 xa = make_float2(u2f(sr[c]), u2f(sr[c + 1])), xb = make_float2(u2f(sr[c + 2]), u2f(sr[c + 3]));
-            const float2 da = HAS_BIAS ? __fadd2_rn(xa, nmp) : __ffma2_rn(xa, kf2, nmp);
-            const float2 db = HAS_BIAS ? __fadd2_rn(xb, nmp) : __ffma2_rn(xb, kf2, nmp);
+            const float2 ya = make_float2(u2f(sr[c]), u2f(sr[c + 1])), yb = make_float2(u2f(sr[c + 2]), u2f(sr[c + 3]));
+            // d = t - m' (one rounding of x * kf - m' without bias)
+            const float2 da = HAS_BIAS ? __fadd2_rn(ya, nmp) : __ffma2_rn(ya, kf2, nmp);
+            const float2 db = HAS_BIAS ? __fadd2_rn(yb, nmp) : __ffma2_rn(yb, kf2, nmp);
             // FP16 mode: 2 of every 8 pairs take the polynomial, the rest the
             // special-function unit (measured: the best split with two
             // softmax warps per SM sub-partition; the FP32 mode, with four,
@@ -477,9 +473,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
             fold_partials(j - 1, alpha_prev);
           } else if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-            for (int i = 0; i < kHalfD / 32; ++i) {
+            for (int i = 0; i < D / 64; ++i) {
               uint32_t o[32];
-              tmem_ld32(t_o + 32 * i, o);
+              tmem_ld16x64b_x32(t_o + 64 * i, o);
               tmem_ld_wait();
 #pragma unroll
               for (int e = 0; e < 32; e += 2) {
@@ -487,7 +483,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
                 o[e] = f2u(v2.x);
                 o[e + 1] = f2u(v2.y);
               }
-              tmem_st32(t_o + 32 * i, o);
+              tmem_st16x64b_x32(t_o + 64 * i, o);
             }
             tmem_st_wait();
           }
@@ -504,15 +500,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         tc_fence_after();
         fold_partials(nt[q] - 1, alpha_prev);
       }
-      if (ok) {
-        // the row sum is the sum of both halves' sums
-        const int jx = nt[q];
-        float* xs = xq + (jx & 1) * 256;
-        xs[h * 128 + r] = l;
-        mbar_arrive(&x_bar[2 * q + (jx & 1)]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&x_bar[2 * q + (jx & 1)], (jx >> 1) & 1, abort_flag))) ok = false;
-        else l = h == 0 ? __fadd_rn(l, xs[128 + r]) : __fadd_rn(xs[r], l);
-      }
+      // the row sum is the sum of both halves' sums (l_0 + l_1 in both threads)
+      const float l_other = __shfl_xor_sync(0xffffffffu, l, 2);
+      l = h == 0 ? __fadd_rn(l, l_other) : __fadd_rn(l_other, l);
       if (!ok) {
         fail(abort_flag, a.err, kErrSoftmax);
       } else {
@@ -521,9 +511,10 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         const float* vs = a.v_scale + (size_t)bh * D + h * kHalfD;
         OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D + h * kHalfD;
 #pragma unroll 1
-        for (int i = 0; i < kHalfD / 32; ++i) {
+        for (int i = 0; i < D / 64; ++i) {
+          // o[e] = channel h d/2 + 32 i + e of this row
           uint32_t o[32];
-          tmem_ld32(t_o + 32 * i, o);
+          tmem_ld16x64b_x32(t_o + 64 * i, o);
           tmem_ld_wait();
           if (row < a.N) {
             uint32_t hh[16];
@@ -638,10 +629,25 @@ __global__ void timeout_probe_kernel(int* err) {
 }
 
 // ------------------------------------------------------------------ launchers
-static bool make_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv) {
+// Q tiles (and the debug tile's K) in row order.
+static bool make_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mq, CUtensorMap* mk) {
   return make_tmap_u8_3d(mq, w.q_codes, pb.d, pb.Npad, pb.BH, pb.d, 128) &&
-         make_tmap_u8_3d(mk, w.k_codes, pb.d, pb.Npad, pb.BH, pb.d, 128) &&
-         (mv == nullptr || make_tmap_u8_3d(mv, w.vt_codes, pb.Npad, pb.d, pb.BH, 128, pb.d));
+         make_tmap_u8_3d(mk, w.k_codes, pb.d, pb.Npad, pb.BH, pb.d, 128);
+}
+
+// The attention kernel's K and V^T tiles in pair order: shared-memory row
+// 2i + e holds key 64e + i of the 128-key tile (K), channel (d/2) e + i (V^T).
+//   K   [BH][Npad][d]: dims (d, e = 2, i = 64, tile, bh), box (d, 2, 64, 1, 1)
+//   V^T [BH][d][Npad]: dims (Npad, e = 2, i = d/2, bh), box (128, 2, d/2, 1)
+static bool make_pair_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mk, CUtensorMap* mv) {
+  const uint64_t D = (uint64_t)pb.d, Np = (uint64_t)pb.Npad;
+  const uint64_t kd[5] = {D, 2, 64, Np / 128, (uint64_t)pb.BH};
+  const uint64_t ks[4] = {64 * D, D, 128 * D, Np * D};
+  const uint32_t kb[5] = {(uint32_t)D, 2, 64, 1, 1};
+  const uint64_t vd[4] = {Np, 2, D / 2, (uint64_t)pb.BH};
+  const uint64_t vs[3] = {(D / 2) * Np, Np, D * Np};
+  const uint32_t vb[4] = {128, 2, (uint32_t)(D / 2), 1};
+  return make_tmap_u8_nd(mk, w.k_codes, 5, kd, ks, kb, (int)D) && make_tmap_u8_nd(mv, w.vt_codes, 4, vd, vs, vb, 128);
 }
 
 template <int D, typename OutT, bool HAS_BIAS, bool F16ACC>
@@ -660,8 +666,8 @@ static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const 
 }
 
 cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
-  if (!make_maps(w, pb, &mq, &mk, &mv)) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, mk_rows;
+  if (!make_maps(w, pb, &mq, &mk_rows) || !make_pair_maps(w, pb, &mk, &mv)) return cudaErrorInvalidValue;
   AttnArgs a;
   a.q_scale = w.q_scale;
   a.k_scale = w.k_scale;
@@ -702,7 +708,7 @@ cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s) {
 cudaError_t launch_debug_qk(const WsPtrs& w, const Problem& pb, int bh, int q_tile, int k_tile, int32_t* out,
                             cudaStream_t s) {
   CUtensorMap mq, mk;
-  if (!make_maps(w, pb, &mq, &mk, nullptr)) return cudaErrorInvalidValue;
+  if (!make_maps(w, pb, &mq, &mk)) return cudaErrorInvalidValue;
   if (pb.d == 128)
     debug_qk_kernel<128><<<1, 128, 0, s>>>(mq, mk, bh, q_tile, k_tile, out, w.error);
   else

@@ -105,5 +105,11 @@ cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s);
 // the swizzle that matches a row of box0 bytes (64 or 128).
 bool make_tmap_u8_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                      uint32_t box0, uint32_t box1);
+// A uint8 tensor of `rank` (2..5) dimensions, dims[0] innermost and
+// contiguous, strides[i] = bytes between consecutive indices of dimension
+// i + 1 (any order: a map may walk rows out of their memory order), a box of
+// box[0..rank) elements; swizzle_bytes 128, 64 or 0.
+bool make_tmap_u8_nd(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                     const uint32_t* box, int swizzle_bytes);
 
 }  // namespace sage

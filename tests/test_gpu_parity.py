@@ -135,6 +135,35 @@ def test_attention_matches_oracle(N, d, dtype, law, smooth_q, causal, mode):
     compare_out(got, ref32, flip, dtype, (N, d, dtype, causal, mode))
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("case", ["zero_k_granules", "zero_q_granule"])
+def test_attention_zero_scale_granules_with_masks(mode, case):
+    """Degenerate scales under causal and ragged masks.  zero_k_granules: K is
+    the same vector for every token, so the smoothed K and every K scale are
+    0 and every logit is 0 (each row averages the V of the keys it sees).
+    zero_q_granule: Q rows 32..63 are 0 (no Q smoothing), so that granule's
+    scale is 0.  Masked keys must stay out in both."""
+    N, d = 300, 128
+    w = small_workload(N, d, "fp16", "k_bias", False, mode, causal=True)
+    q, k, v = [t.clone() for t in inputs.generate(w)]
+    if case == "zero_k_granules":
+        k[:] = k[:, :, :1, :]
+    else:
+        q[:, :, 32:64, :] = 0
+    q, k, v = [t.cuda() for t in (q, k, v)]
+    B, H = 1, 2
+    ws = api.alloc_workspace(B, H, N, d, mode)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, True, mode, 0, False, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    oz = oracle_quant((q, k, v), mode, False)
+    if case == "zero_k_granules":
+        assert not np.any(oz["k_scale"])
+    ref32, flip = orc.attention_int8_fp8(oz, True, with_flip=True)
+    got = out.float().cpu().reshape(B * H, N, d).numpy()
+    compare_out(got, ref32, flip, "fp16", (case, mode))
+
+
 def test_full_size_llm_prefill_sampled_rows():
     """The B1 H32 N8192 d128 bf16 causal workload at full size, in the launch
     configuration the bench times: quantization bit-exact everywhere, the
