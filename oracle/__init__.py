@@ -237,11 +237,13 @@ def qk_s32(qc: np.ndarray, kc: np.ndarray) -> np.ndarray:
     return out
 
 
-def quantize_int8_fp8(q, k, v, smooth_q: bool, mode: int) -> dict:
+def quantize_int8_fp8(q, k, v, smooth_q: bool, mode: int, Vr: float | None = None) -> dict:
     """The whole preprocessing of the INT8/FP8 modes for [BH, N, d] inputs:
-    K smoothing, optional Q smoothing with its bias, INT8 Q/K, FP8 V."""
+    K smoothing, optional Q smoothing with its bias, INT8 Q/K, FP8 V (range
+    Vr: the mode's default unless given)."""
     q, k, v = _f32(q), _f32(k), _f32(v)
-    Vr = VR_F16ACC if mode == MODE_INT8_FP8_F16ACC else VR_FP32ACC
+    if Vr is None:
+        Vr = VR_F16ACC if mode == MODE_INT8_FP8_F16ACC else VR_FP32ACC
     mean_k = channel_mean(k)
     mean_q = channel_mean(q) if smooth_q else None
     amax_v = channel_absmax(v)
@@ -254,17 +256,22 @@ def quantize_int8_fp8(q, k, v, smooth_q: bool, mode: int) -> dict:
                 N=q.shape[1], d=q.shape[2], mode=mode)
 
 
-def attention_int8_fp8(qz: dict, causal: bool, rows=None, with_flip: bool = False):
+def attention_int8_fp8(qz: dict, causal: bool, rows=None, with_flip: bool = False, Pr: float | None = None,
+                       chunk: int = 64):
     """Tiled online-softmax attention on quantized inputs.  rows: None (all)
     or an int array of query rows (same rows for every slice).
     Returns float32 [BH, nrows, d] before the cast to the output dtype; with
     `with_flip`, also the per-element change one P~ code moved to a
-    neighbouring code would cause (a sensitivity figure for comparisons)."""
+    neighbouring code would cause (a sensitivity figure for comparisons).
+    Pr: the P~ range (the mode's default unless given); chunk: keys per FP16
+    partial in the FP16-accumulator mode (64, or 32 without delayed
+    buffering)."""
     qc, kc, vt = qz["q_codes"], qz["k_codes"], qz["vt_codes"]
     BH, Np, d = qc.shape
     N = qz["N"]
     mode = qz["mode"]
-    Pr = PR_F16ACC if mode == MODE_INT8_FP8_F16ACC else PR_FP32ACC
+    if Pr is None:
+        Pr = PR_F16ACC if mode == MODE_INT8_FP8_F16ACC else PR_FP32ACC
     if rows is None:
         r = None
         nrows = N
@@ -275,8 +282,59 @@ def attention_int8_fp8(qz: dict, causal: bool, rows=None, with_flip: bool = Fals
     flip = np.empty((BH, nrows, d), np.float32) if with_flip else None
     bias = qz["q_bias"]
     lib().orc_attn_int8_fp8(_p(qc), _p(qz["q_scale"]), _p(kc), _p(qz["k_scale"]), _p(vt),
-                            _p(qz["v_scale"]), _p(bias), BH, N, Np, d, int(causal), int(mode),
-                            ctypes.c_float(qz.get("Pr", Pr)), _p(r), nrows, _p(out), _p(flip))
+                            _p(qz["v_scale"]), _p(bias), BH, N, Np, d, int(causal), int(mode), int(chunk),
+                            ctypes.c_float(Pr), _p(r), nrows, _p(out), _p(flip))
+    return (out, flip) if with_flip else out
+
+
+def quantize_int8_fp8_gqa(q, k, v, smooth_q: bool, mode: int, Vr: float | None = None) -> dict:
+    """Preprocessing with grouped key/value heads and separate lengths: q
+    [B, Hq, Nq, d], k and v [B, Hkv, Nk, d].  Each tensor is smoothed and
+    quantized per its own heads and tokens as in quantize_int8_fp8; the
+    Q-smoothing bias of query head hq is mean_q(hq) . k~ over the keys of its
+    key/value head hq / G, G = Hq / Hkv."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    G = Hq // Hkv
+    if Vr is None:
+        Vr = VR_F16ACC if mode == MODE_INT8_FP8_F16ACC else VR_FP32ACC
+    qf, kf, vf = q.reshape(B * Hq, Nq, d), k.reshape(B * Hkv, Nk, d), v.reshape(B * Hkv, Nk, d)
+    mean_k = channel_mean(kf)
+    mean_q = channel_mean(qf) if smooth_q else None
+    qc, sq = quant_int8(qf, mean_q, Q_GRANULE)
+    kc, sk = quant_int8(kf, mean_k, K_GRANULE)
+    vt, sv = quant_v_fp8(vf, channel_absmax(vf), Vr)
+    bias = None
+    if smooth_q:
+        # each query head against its key/value head's keys
+        kx = np.repeat(kf.reshape(B, Hkv, Nk, d), G, axis=1).reshape(B * Hq, Nk, d)
+        mkx = np.repeat(mean_k.reshape(B, Hkv, d), G, axis=1).reshape(B * Hq, d)
+        bias = q_bias(kx, mkx, mean_q)
+    return dict(q_codes=qc, q_scale=sq, k_codes=kc, k_scale=sk, vt_codes=vt, v_scale=sv, k_mean=mean_k,
+                q_mean=mean_q, q_bias=bias, B=B, Hq=Hq, Hkv=Hkv, Nq=Nq, Nk=Nk, d=d, mode=mode)
+
+
+def attention_int8_fp8_gqa(qz: dict, causal: bool, rows=None, with_flip: bool = False, Pr: float | None = None,
+                           chunk: int = 64):
+    """Attention on quantize_int8_fp8_gqa's output: query head hq reads
+    key/value head hq / G; causal rows see keys j <= i + (Nk - Nq).
+    Returns float32 [B*Hq, nrows, d] (and the P~ sensitivity with with_flip)."""
+    B, Hq, Hkv, Nq, Nk, d = qz["B"], qz["Hq"], qz["Hkv"], qz["Nq"], qz["Nk"], qz["d"]
+    mode = qz["mode"]
+    if Pr is None:
+        Pr = PR_F16ACC if mode == MODE_INT8_FP8_F16ACC else PR_FP32ACC
+    if rows is None:
+        r, nrows = None, Nq
+    else:
+        r = np.ascontiguousarray(rows, np.int32)
+        nrows = len(r)
+    out = np.empty((B * Hq, nrows, d), np.float32)
+    flip = np.empty((B * Hq, nrows, d), np.float32) if with_flip else None
+    lib().orc_attn_int8_fp8_gqa(_p(qz["q_codes"]), _p(qz["q_scale"]), _p(qz["k_codes"]), _p(qz["k_scale"]),
+                                _p(qz["vt_codes"]), _p(qz["v_scale"]), _p(qz["q_bias"]), B, Hq, Hkv, Nq, Nk,
+                                npad(Nq), npad(Nk), d, int(causal), int(mode), int(chunk), ctypes.c_float(Pr),
+                                _p(r), nrows, _p(out), _p(flip))
     return (out, flip) if with_flip else out
 
 
@@ -341,17 +399,20 @@ def nvfp4_block(x, g: float):
 # Plain definitions: unquantized attention and the accuracy metrics.
 # --------------------------------------------------------------------------
 def attention_fp64(q, k, v, causal: bool, rows=None) -> np.ndarray:
-    """softmax(Q K^T / sqrt(d)) V in float64, [BH, N, d] inputs."""
+    """softmax(Q K^T / sqrt(d)) V in float64.  q [BH, Nq, d], k and v
+    [BH, Nk, d] (Nq may differ from Nk; a causal row i sees keys
+    j <= i + Nk - Nq)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
-    BH, N, d = q.shape
-    idx = np.arange(N) if rows is None else np.asarray(rows)
+    BH, Nq, d = q.shape
+    Nk = k.shape[1]
+    idx = np.arange(Nq) if rows is None else np.asarray(rows)
     out = np.empty((BH, len(idx), d), np.float64)
     for bh in range(BH):
         s = q[bh, idx] @ k[bh].T / np.sqrt(d)
         if causal:
-            s = np.where(np.arange(N)[None, :] <= idx[:, None], s, -np.inf)
+            s = np.where(np.arange(Nk)[None, :] <= idx[:, None] + (Nk - Nq), s, -np.inf)
         s = s - s.max(axis=1, keepdims=True)
         p = np.exp(s)
         out[bh] = (p / p.sum(axis=1, keepdims=True)) @ v[bh]

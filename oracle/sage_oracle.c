@@ -355,7 +355,9 @@ static double e4m3_step(int cm)
  *   FP32 accumulator: acc_c = alpha * acc_c + fl32(exact sum_j P~_j v^_jc)
  *   FP16 accumulator (SageAttention2++ Sec. 3.2): per 64-key chunk,
  *        h = f16(exact sum of its first 32 products), h = f16(h + exact sum of
- *        the next 32); acc_c = (alpha * acc_c + h_chunk0) + h_chunk1
+ *        the next 32); acc_c = (alpha * acc_c + h_chunk0) + h_chunk1.  With
+ *        chunk = 32 (the accuracy sweep's other depth: no delayed buffering)
+ *        each 32-key sum is rounded to f16 and added to the fp32 value alone.
  *   O_ic  = acc_c * scale_v[c] / (Pr * l)
  * exp2 is orc_exp2 above.  Masked keys (j >= N, or j > i when causal) take no
  * part.  The exact sums of e4m3 products fit a double: each product has 8
@@ -368,14 +370,15 @@ static double e4m3_step(int cm)
  * with implementations whose exponential differs in the last bits. */
 static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* vt,
                      float sq, const float* sk, const float* bias, const float* scale_v,
-                     int N, int Npad, int d, int causal, int mode, float Pr,
+                     int N, int Npad, int d, int causal, int koff, int mode, int chunk, float Pr,
                      float* acc, double* fl, float* tvals, int* pcode, float* out_row,
                      float* flip_row)
 {
   const float c_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   float m = -INFINITY, l = 0.0f;
   for (int c = 0; c < d; ++c) { acc[c] = 0.0f; fl[c] = 0.0; }
-  int jmax = causal ? (i < N - 1 ? i : N - 1) : N - 1;   /* last visible key */
+  /* last visible key: all N keys, or (causal) keys j <= i + koff */
+  int jmax = causal ? (i + koff < N - 1 ? i + koff : N - 1) : N - 1;
   for (int j0 = 0; j0 <= jmax; j0 += 128) {
     float mt = -INFINITY;
     for (int j = j0; j < j0 + 128; ++j) {
@@ -414,14 +417,14 @@ static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* v
         acc[c] = alpha * acc[c] + (float)sum;
       } else {
         float a = alpha * acc[c];
-        for (int ch = 0; ch < 128; ch += 64) {
+        for (int ch = 0; ch < 128; ch += chunk) {
           double s0 = 0.0, s1 = 0.0;
           for (int j = ch; j < ch + 32; ++j)
             if (pcode[j] >= 0) s0 += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
-          for (int j = ch + 32; j < ch + 64; ++j)
+          for (int j = ch + 32; j < ch + chunk; ++j)
             if (pcode[j] >= 0) s1 += orc_e4m3_decode(pcode[j]) * orc_e4m3_decode(vrow[j]);
           double h = orc_f16_round(s0);
-          h = orc_f16_round(h + s1);
+          if (chunk == 64) h = orc_f16_round(h + s1);
           a = a + (float)h;
         }
         acc[c] = a;
@@ -436,15 +439,57 @@ static void attn_row(int i, const int8_t* qc, const int8_t* kc, const uint8_t* v
   }
 }
 
+/* Attention with grouped key/value heads and separate query and key lengths.
+ * Query head hq of batch b reads key/value head hq / G, G = Hq / Hkv (G = 1:
+ * every head its own; Hkv = 1: one shared head).  Nq query rows, Nk keys;
+ * a causal mask lets row i see keys j <= i + (Nk - Nq) (the last query row
+ * sees every key; Nq == Nk is the usual j <= i).  Layouts:
+ *   qc [B*Hq, Npq, d], sq [B*Hq, Npq/32], bias [B*Hq, Npk] (or NULL)
+ *   kc [B*Hkv, Npk, d], sk [B*Hkv, Npk/64], vt [B*Hkv, d, Npk], scale_v [B*Hkv, d]
+ * rows == NULL means all Nq rows.  out, flip: [B*Hq, nrows, d] (flip may be
+ * NULL).  chunk: keys per FP16 partial in the FP16-accumulator mode. */
+ORC_EXPORT void orc_attn_int8_fp8_gqa(const int8_t* qc, const float* sq, const int8_t* kc,
+                                      const float* sk, const uint8_t* vt, const float* scale_v,
+                                      const float* bias, int B, int Hq, int Hkv, int Nq, int Nk,
+                                      int Npq, int Npk, int d, int causal, int mode, int chunk,
+                                      float Pr, const int* rows, int nrows, float* out, float* flip)
+{
+  if (chunk != 32) chunk = 64;
+  init_tables();
+  const int BH = B * Hq, G = Hq / Hkv, koff = Nk - Nq;
+#pragma omp parallel
+  {
+    float* acc = (float*)malloc(sizeof(float) * d);
+    double* fl = (double*)malloc(sizeof(double) * d);
+    float* tv = (float*)malloc(sizeof(float) * 128);
+    int* pc = (int*)malloc(sizeof(int) * 128);
+#pragma omp for schedule(dynamic, 4) collapse(2)
+    for (int bh = 0; bh < BH; ++bh)
+      for (int r = 0; r < nrows; ++r) {
+        int i = rows ? rows[r] : r;
+        const int bkv = (bh / Hq) * Hkv + (bh % Hq) / G;
+        const size_t o = ((size_t)bh * nrows + r) * d;
+        attn_row(i, qc + (size_t)bh * Npq * d, kc + (size_t)bkv * Npk * d,
+                 vt + (size_t)bkv * d * Npk, sq[(size_t)bh * (Npq / 32) + i / 32],
+                 sk + (size_t)bkv * (Npk / 64), bias ? bias + (size_t)bh * Npk : NULL,
+                 scale_v + (size_t)bkv * d, Nk, Npk, d, causal, koff, mode, chunk, Pr, acc, fl, tv,
+                 pc, out + o, flip ? flip + o : NULL);
+      }
+    free(acc); free(fl); free(tv); free(pc);
+  }
+}
+
 /* Attention output for the listed query rows of every (b,h) slice.
  * rows == NULL means all N rows (then nrows must be N).  out: [BH, nrows, d].
+ * chunk: keys per FP16 partial in the FP16-accumulator mode (64, or 32).
  * flip (may be NULL): [BH, nrows, d] single-code sensitivity (see attn_row). */
 ORC_EXPORT void orc_attn_int8_fp8(const int8_t* qc, const float* sq, const int8_t* kc,
                                   const float* sk, const uint8_t* vt, const float* scale_v,
                                   const float* bias, int BH, int N, int Npad, int d,
-                                  int causal, int mode, float Pr, const int* rows, int nrows,
-                                  float* out, float* flip)
+                                  int causal, int mode, int chunk, float Pr, const int* rows,
+                                  int nrows, float* out, float* flip)
 {
+  if (chunk != 32) chunk = 64;
   init_tables();
 #pragma omp parallel
   {
@@ -460,7 +505,7 @@ ORC_EXPORT void orc_attn_int8_fp8(const int8_t* qc, const float* sq, const int8_
         attn_row(i, qc + (size_t)bh * Npad * d, kc + (size_t)bh * Npad * d,
                  vt + (size_t)bh * d * Npad, sq[(size_t)bh * (Npad / 32) + i / 32],
                  sk + (size_t)bh * (Npad / 64), bias ? bias + (size_t)bh * Npad : NULL,
-                 scale_v + (size_t)bh * d, N, Npad, d, causal, mode, Pr, acc, fl, tv, pc,
+                 scale_v + (size_t)bh * d, N, Npad, d, causal, 0, mode, chunk, Pr, acc, fl, tv, pc,
                  out + o, flip ? flip + o : NULL);
       }
     free(acc); free(fl); free(tv); free(pc);

@@ -8,14 +8,15 @@ import pytest
 
 import oracle as orc
 import test_oracle as t1
+import test_oracle_gqa as t3
 import test_oracle_pins2 as t2
 
 PLANTS = {
     # FP16 accumulator: one rounding of the whole 64-key sum (no delayed buffer)
-    "f16_single_rounding": [("          double h = orc_f16_round(s0);\n          h = orc_f16_round(h + s1);",
+    "f16_single_rounding": [("          double h = orc_f16_round(s0);\n          if (chunk == 64) h = orc_f16_round(h + s1);",
                              "          double h = orc_f16_round(s0 + s1);")],
     # FP16 accumulator: each 32-key MMA result flushed to fp32 on its own
-    "f16_flush_every_32": [("          double h = orc_f16_round(s0);\n          h = orc_f16_round(h + s1);",
+    "f16_flush_every_32": [("          double h = orc_f16_round(s0);\n          if (chunk == 64) h = orc_f16_round(h + s1);",
                             "          a = a + (float)orc_f16_round(s0);\n          double h = orc_f16_round(s1);")],
     # NVFP4 block scale against the wrong e2m1 range (4 instead of 6)
     "fp4_scale_range": [("bs = orc_ue4m3_encode((double)(a / (6.0f * g)));",
@@ -38,6 +39,12 @@ PLANTS = {
                    "      if (bias) deq = deq - bias[j];\n      const float t = deq * c_log2;\n      tvals[j - j0] = t;\n"
                    "      if (t > mt) mt = t;\n    }\n    const float m_new = m > mt ? m : mt;\n    const float alpha = "
                    "orc_exp2(m - m_new);   /* first tile")],
+    # grouped heads: query head read against the wrong key/value head
+    "gqa_head_map": [("const int bkv = (bh / Hq) * Hkv + (bh % Hq) / G;",
+                      "const int bkv = (bh / Hq) * Hkv + (bh % Hq) % Hkv;")],
+    # separate lengths: causal mask aligned at the top left instead of the bottom right
+    "cross_causal_offset": [("const int BH = B * Hq, G = Hq / Hkv, koff = Nk - Nq;",
+                             "const int BH = B * Hq, G = Hq / Hkv, koff = 0;")],
     # P~ quantized without its range factor Pr
     "p_without_range": [("pcode[j] = (j0 + j <= jmax) ? orc_e4m3_encode((double)(p * Pr)) : -1;",
                          "pcode[j] = (j0 + j <= jmax) ? orc_e4m3_encode((double)p) : -1;")],
@@ -62,6 +69,8 @@ CATCHERS = {
     "no_rescale": t1.test_dropping_the_rescale_is_caught,
     "k_granule_index": t1.test_dropping_the_rescale_is_caught,
     "bias_sign": lambda: t1.test_multi_tile_ragged_close_to_fp64(orc.MODE_INT8_FP8),
+    "gqa_head_map": t3.check_gqa_equals_repeated_heads,
+    "cross_causal_offset": t3.check_cross_length_causal,
     "p_without_range": lambda: t1.test_quantized_attention_close_to_fp64(orc.MODE_INT8_FP8, False),
 }
 
