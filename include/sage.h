@@ -177,6 +177,37 @@ SAGE_API sage_status sage_attn_fwd_ranges(const void* q, const void* k, const vo
                                           int N, int d, int causal, int mode, int dtype, int smooth_q, float Pr,
                                           float Vr, void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* Grouped key/value heads and separate query and key lengths (decoding or
+ * chunked prefill against a longer key cache, cross-attention, and models whose
+ * query heads share key/value heads).  The pages' method per query head
+ * (SageAttention2 abstract; SageAttention2++ summary Sec. 2, 2.1, 3) with:
+ *   q, out [B, Hq, Nq, d]; k, v [B, Hkv, Nk, d]; Hq a multiple of Hkv; query
+ *   head h reads key/value head h / (Hq / Hkv);
+ *   K smoothed per key/value head over its Nk tokens, V scaled per channel of
+ *   its key/value head, Q quantized per query head (smoothed with smooth_q,
+ *   the bias mean_q(h) . k~ over the keys of h's key/value head);
+ *   causal: query row i sees keys j <= i + Nk - Nq (the last query row sees
+ *   all keys; needs Nq <= Nk, else SAGE_ERR_UNSUPPORTED).
+ * INT8/FP8 modes only (SAGE_MODE_NVFP4 needs Hq == Hkv and Nq == Nk).  With
+ * Hq == Hkv and Nq == Nk these are the per-head entry points above, with the
+ * same workspace layout.  Workspace layout (sage_workspace_layout_gqa):
+ * q_codes [B*Hq, Npq, d], q_scale [B*Hq, Npq/32], q_mean [B*Hq, d], q_bias
+ * [B*Hq, Npk]; k_codes [B*Hkv, Npk, d], vt_codes [B*Hkv, d, Npk], k_scale
+ * [B*Hkv, Npk/64], v_scale and k_mean [B*Hkv, d]; Npq, Npk = Nq, Nk rounded
+ * up to 128.  Other arguments, alignment and error behaviour as for the
+ * per-head calls. */
+SAGE_API sage_status sage_workspace_layout_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode,
+                                               sage_ws_layout* out);
+SAGE_API sage_status sage_quantize_qkv_gqa(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                                           int Hkv, int Nq, int Nk, int d, int smooth_q, int mode, void* ws,
+                                           size_t ws_bytes, sage_stream_t stream);
+SAGE_API sage_status sage_attn_quantized_gqa(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int Hq,
+                                             int Hkv, int Nq, int Nk, int d, int causal, int smooth_q, int mode,
+                                             sage_stream_t stream);
+SAGE_API sage_status sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                                       int Nq, int Nk, int d, int causal, int mode, int dtype, int smooth_q, void* ws,
+                                       size_t ws_bytes, sage_stream_t stream);
+
 /* Parity helper: the INT32 tile S = Q^ K^T of query tile `q_tile` and key tile
  * `k_tile` (128 x 128) of slice `bh`, computed by the same tensor-core path as
  * the attention kernel (kind::i8 MMA, accumulator in TMEM).  out: device

@@ -21,7 +21,8 @@ DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
 
 EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_quantize_qkv_static",
             "sage_attn_quantized",
-            "sage_attn_fwd", "sage_attn_fwd_ranges", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_probe_mma_rate",
+            "sage_attn_fwd", "sage_attn_fwd_ranges", "sage_workspace_layout_gqa", "sage_quantize_qkv_gqa",
+            "sage_attn_quantized_gqa", "sage_attn_fwd_gqa", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_probe_mma_rate",
             "sage_check", "sage_last_error")
 PROBE_I8, PROBE_F8_F32ACC, PROBE_F8_F16ACC, PROBE_BF16, PROBE_FP4 = range(5)
 
@@ -65,6 +66,14 @@ def lib() -> ctypes.CDLL:
         f = ctypes.c_float
         L.sage_attn_fwd_ranges.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, vp, sz, vp]
         L.sage_attn_fwd_ranges.restype = i
+        L.sage_workspace_layout_gqa.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(WsLayout)]
+        L.sage_workspace_layout_gqa.restype = i
+        L.sage_quantize_qkv_gqa.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_quantize_qkv_gqa.restype = i
+        L.sage_attn_quantized_gqa.argtypes = [vp, sz, vp, i, i, i, i, i, i, i, i, i, i, vp]
+        L.sage_attn_quantized_gqa.restype = i
+        L.sage_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_attn_fwd_gqa.restype = i
         L.sage_debug_qk_s32.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
         L.sage_debug_qk_s32.restype = i
         L.sage_debug_fp4_s.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
@@ -133,6 +142,57 @@ def sage_attn_fwd_ranges(q, k, v, out, B, H, N, d, causal, mode, dtype, smooth_q
                          stream=None):
     _raise(lib().sage_attn_fwd_ranges(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, int(causal), mode, dtype,
                                       int(smooth_q), float(Pr), float(Vr), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def sage_workspace_layout_gqa(B, Hq, Hkv, Nq, Nk, d, mode) -> WsLayout:
+    out = WsLayout()
+    _raise(lib().sage_workspace_layout_gqa(B, Hq, Hkv, Nq, Nk, d, mode, ctypes.byref(out)))
+    return out
+
+
+def sage_quantize_qkv_gqa(q, k, v, dtype, B, Hq, Hkv, Nq, Nk, d, smooth_q, mode, ws, ws_bytes, stream=None):
+    _raise(lib().sage_quantize_qkv_gqa(_ptr(q), _ptr(k), _ptr(v), dtype, B, Hq, Hkv, Nq, Nk, d, int(smooth_q), mode,
+                                       _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def sage_attn_quantized_gqa(ws, ws_bytes, out, dtype, B, Hq, Hkv, Nq, Nk, d, causal, smooth_q, mode, stream=None):
+    _raise(lib().sage_attn_quantized_gqa(_ptr(ws), ws_bytes, _ptr(out), dtype, B, Hq, Hkv, Nq, Nk, d, int(causal),
+                                         int(smooth_q), mode, _stream(stream)))
+
+
+def sage_attn_fwd_gqa(q, k, v, out, B, Hq, Hkv, Nq, Nk, d, causal, mode, dtype, smooth_q, ws, ws_bytes, stream=None):
+    _raise(lib().sage_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, Nq, Nk, d, int(causal), mode,
+                                   dtype, int(smooth_q), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def alloc_workspace_gqa(B, Hq, Hkv, Nq, Nk, d, mode, device="cuda") -> torch.Tensor:
+    """Device workspace for the grouped-head / separate-length calls (1024-byte aligned)."""
+    n = sage_workspace_layout_gqa(B, Hq, Hkv, Nq, Nk, d, mode).total
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 1024
+    return raw[off:off + n]
+
+
+def ws_views_gqa(ws: torch.Tensor, B, Hq, Hkv, Nq, Nk, d, mode) -> dict:
+    """Typed views of the quantized buffers of a grouped-head workspace (INT8/FP8)."""
+    L = sage_workspace_layout_gqa(B, Hq, Hkv, Nq, Nk, d, mode)
+    BHq, BHk = B * Hq, B * Hkv
+    Npq, Npk = (Nq + 127) // 128 * 128, (Nk + 127) // 128 * 128
+
+    def view(off, nbytes, dtype, shape):
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    return dict(
+        q_codes=view(L.q_codes, BHq * Npq * d, torch.int8, (BHq, Npq, d)),
+        k_codes=view(L.k_codes, BHk * Npk * d, torch.int8, (BHk, Npk, d)),
+        vt_codes=view(L.vt_codes, BHk * d * Npk, torch.uint8, (BHk, d, Npk)),
+        q_scale=view(L.q_scale, BHq * (Npq // 32) * 4, torch.float32, (BHq, Npq // 32)),
+        k_scale=view(L.k_scale, BHk * (Npk // 64) * 4, torch.float32, (BHk, Npk // 64)),
+        v_scale=view(L.v_scale, BHk * d * 4, torch.float32, (BHk, d)),
+        k_mean=view(L.k_mean, BHk * d * 4, torch.float32, (BHk, d)),
+        q_mean=view(L.q_mean, BHq * d * 4, torch.float32, (BHq, d)),
+        q_bias=view(L.q_bias, BHq * Npk * 4, torch.float32, (BHq, Npk)),
+    )
 
 
 def sage_debug_qk_s32(ws, ws_bytes, B, H, N, d, bh, q_tile, k_tile, out, stream=None):

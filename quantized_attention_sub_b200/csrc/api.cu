@@ -34,10 +34,34 @@ sage_status check_shape(int B, int H, int N, int d, int mode) {
   return SAGE_OK;
 }
 
-sage_ws_layout layout_of(int B, int H, int N, int d, int mode) {
+// Grouped key/value heads (Hq query heads per batch, Hkv key/value heads,
+// Hq % Hkv == 0) and separate query / key lengths.  INT8/FP8 modes only
+// unless the shapes coincide (then the per-head checks and layout apply).
+sage_status check_shape_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1)
+    return set_err(SAGE_ERR_INVALID_ARG, "B, Hq, Hkv, Nq and Nk must be >= 1%s");
+  if (Hq % Hkv) return set_err(SAGE_ERR_INVALID_ARG, "Hq must be a multiple of Hkv%s");
+  sage_status st = check_shape(B, Hq, Nq, d, mode);
+  if (st != SAGE_OK) return st;
+  if ((st = check_shape(B, Hkv, Nk, d, mode)) != SAGE_OK) return st;
+  if (mode == SAGE_MODE_NVFP4 && (Hq != Hkv || Nq != Nk))
+    return set_err(SAGE_ERR_UNSUPPORTED, "the NVFP4 mode needs Hq == Hkv and Nq == Nk%s");
+  const long long npk = ((long long)Nk + 127) / 128 * 128;
+  if ((long long)B * Hq * npk >= (1LL << 31))
+    return set_err(SAGE_ERR_UNSUPPORTED, "problem too large (B*Hq*Npad_k must be < 2^31)%s");
+  return SAGE_OK;
+}
+
+sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode);
+
+sage_ws_layout layout_of(int B, int H, int N, int d, int mode) { return layout_of_gqa(B, H, H, N, N, d, mode); }
+
+sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode) {
   sage_ws_layout L;
   memset(&L, 0, sizeof(L));
-  const size_t BH = (size_t)B * H, Np = ((size_t)N + 127) / 128 * 128;
+  const bool split = Hq != Hkv || Nq != Nk;
+  const size_t BH = (size_t)B * Hq, Np = ((size_t)Nq + 127) / 128 * 128;
+  const size_t BHk = (size_t)B * Hkv, Npk = ((size_t)Nk + 127) / 128 * 128;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -55,18 +79,20 @@ sage_ws_layout layout_of(int B, int H, int N, int d, int mode) {
     L.global_scale = take(BH * 4 * sizeof(float));
   } else {
     L.q_codes = take(BH * Np * d);
-    L.k_codes = take(BH * Np * d);
-    L.vt_codes = take(BH * d * Np);
+    L.k_codes = take(BHk * Npk * d);
+    L.vt_codes = take(BHk * d * Npk);
     L.q_scale = take(BH * (Np / 32) * sizeof(float));
-    L.k_scale = take(BH * (Np / 64) * sizeof(float));
-    L.v_scale = take(BH * d * sizeof(float));
+    L.k_scale = take(BHk * (Npk / 64) * sizeof(float));
+    L.v_scale = take(BHk * d * sizeof(float));
     L.global_scale = take(0);
   }
-  L.k_mean = take(BH * d * sizeof(float));
+  L.k_mean = take(BHk * d * sizeof(float));
   L.q_mean = take(BH * d * sizeof(float));
-  L.q_bias = take(BH * Np * sizeof(float));
+  L.q_bias = take(BH * Npk * sizeof(float));
   // statistics partials and V multipliers of the quantize pass
-  L.scratch = take(sage::quant_scratch_floats((int)BH, (int)Np, d, mode) * sizeof(float));
+  L.scratch = take((split ? sage::quant_scratch_floats_split((int)BH, (int)Np, (int)BHk, (int)Npk, d)
+                          : sage::quant_scratch_floats((int)BH, (int)Np, d, mode)) *
+                   sizeof(float));
   L.total = off;
   return L;
 }
@@ -306,6 +332,84 @@ sage_status sage_attn_fwd_ranges(const void* q, const void* k, const void* v, vo
   st = quantize(q, k, v, dtype, B, H, N, d, smooth_q, mode, Vr, ws, ws_bytes, stream);
   if (st != SAGE_OK) return st;
   return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, Pr, stream, true);
+}
+
+sage_status sage_workspace_layout_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode, sage_ws_layout* out) {
+  sage_status st = check_shape_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  if (st != SAGE_OK) return st;
+  if (!out) return set_err(SAGE_ERR_INVALID_ARG, "layout pointer is null%s");
+  *out = layout_of_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  return SAGE_OK;
+}
+
+static sage::Problem problem_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int dtype, int smooth_q, int mode,
+                                 int causal) {
+  sage::Problem pb{B * Hq, Nq, (Nq + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
+  pb.Hq = Hq;
+  pb.G = Hq / Hkv;
+  pb.Nk = Nk;
+  pb.Npad_k = (Nk + 127) / 128 * 128;
+  return pb;
+}
+
+sage_status sage_quantize_qkv_gqa(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
+                                  int Nq, int Nk, int d, int smooth_q, int mode, void* ws, size_t ws_bytes,
+                                  sage_stream_t stream) {
+  sage_status st = check_shape_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  if (st != SAGE_OK) return st;
+  if (Hq == Hkv && Nq == Nk) return sage_quantize_qkv(q, k, v, dtype, B, Hq, Nq, d, smooth_q, mode, ws, ws_bytes, stream);
+  if (!q || !k || !v) return set_err(SAGE_ERR_INVALID_ARG, "null input pointer%s");
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
+  if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
+    return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
+  const sage_ws_layout L = layout_of_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SAGE_OK) return st;
+  const sage::Problem pb = problem_gqa(B, Hq, Hkv, Nq, Nk, d, dtype, smooth_q, mode, 0);
+  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_quant_split(q, k, v, pb, default_vr(mode), resolve(ws, L), (cudaStream_t)stream),
+                     "quantize launch");
+}
+
+static sage_status attn_quantized_gqa(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int Hq, int Hkv,
+                                      int Nq, int Nk, int d, int causal, int smooth_q, int mode,
+                                      sage_stream_t stream, bool after_quantize) {
+  sage_status st = check_shape_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  if (st != SAGE_OK) return st;
+  if (Hq == Hkv && Nq == Nk)
+    return attn_quantized(ws, ws_bytes, out, dtype, B, Hq, Nq, d, causal, smooth_q, mode, default_pr(mode), stream,
+                          after_quantize);
+  if (causal && Nq > Nk)
+    return set_err(SAGE_ERR_UNSUPPORTED, "a causal mask with Nq > Nk leaves query rows without keys%s");
+  if (!out) return set_err(SAGE_ERR_INVALID_ARG, "null output pointer%s");
+  if (((uintptr_t)out) % 16) return set_err(SAGE_ERR_INVALID_ARG, "output must be 16-byte aligned%s");
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
+  const sage_ws_layout L = layout_of_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  if ((st = check_ws(ws, ws_bytes, L.scratch)) != SAGE_OK) return st;
+  const sage::Problem pb = problem_gqa(B, Hq, Hkv, Nq, Nk, d, dtype, smooth_q, mode, causal);
+  if (!after_quantize &&
+      (st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_attn_i8f8(resolve(const_cast<void*>(ws), L), out, pb, default_pr(mode),
+                                            (cudaStream_t)stream),
+                     "attention launch");
+}
+
+sage_status sage_attn_quantized_gqa(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int Hq, int Hkv,
+                                    int Nq, int Nk, int d, int causal, int smooth_q, int mode, sage_stream_t stream) {
+  return attn_quantized_gqa(ws, ws_bytes, out, dtype, B, Hq, Hkv, Nq, Nk, d, causal, smooth_q, mode, stream, false);
+}
+
+sage_status sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Nq,
+                              int Nk, int d, int causal, int mode, int dtype, int smooth_q, void* ws, size_t ws_bytes,
+                              sage_stream_t stream) {
+  sage_status st = check_shape_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
+  if (st != SAGE_OK) return st;
+  if (causal && Nq > Nk)
+    return set_err(SAGE_ERR_UNSUPPORTED, "a causal mask with Nq > Nk leaves query rows without keys%s");
+  st = sage_quantize_qkv_gqa(q, k, v, dtype, B, Hq, Hkv, Nq, Nk, d, smooth_q, mode, ws, ws_bytes, stream);
+  if (st != SAGE_OK) return st;
+  return attn_quantized_gqa(ws, ws_bytes, out, dtype, B, Hq, Hkv, Nq, Nk, d, causal, smooth_q, mode, stream, true);
 }
 
 sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,

@@ -86,7 +86,9 @@ struct AttnArgs {
   const float* bias;  // null unless smooth_q
   void* out;
   int* err;
-  int N, Npad, causal, num_qblocks;
+  int N, Npad, causal, num_qblocks;     // query rows (padded), causal flag, CTAs per slice
+  int Nk, Npad_k, koff;                 // keys (padded); causal: row i sees keys j <= i + koff
+  int Hq, G;                            // query heads per batch, query heads per key/value head
   int grouped;  // grid (G, query blocks, B*H/G) instead of (query blocks, B*H)
   float c_log2, log2Pr;
 };
@@ -101,6 +103,21 @@ enum : int {
 };
 
 SAGE_DEV float lo_half_to_float(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu))); }
+
+// The CTA's query slice and its key/value slice, read from the special
+// registers each time (volatile: recomputed where used rather than held in
+// registers across the key-tile loop).
+SAGE_DEV int query_slice(const AttnArgs& a) {
+  uint32_t x, y, z, nx;
+  asm volatile("mov.u32 %0, %%ctaid.x;" : "=r"(x));
+  asm volatile("mov.u32 %0, %%ctaid.y;" : "=r"(y));
+  asm volatile("mov.u32 %0, %%ctaid.z;" : "=r"(z));
+  asm volatile("mov.u32 %0, %%nctaid.x;" : "=r"(nx));
+  return a.grouped ? (int)(z * nx + x) : (int)y;
+}
+SAGE_DEV int kv_slice(const AttnArgs& a, int bh) {
+  return a.G == 1 ? bh : (bh / a.Hq) * (a.Hq / a.G) + (bh % a.Hq) / a.G;
+}
 
 }  // namespace
 
@@ -141,13 +158,15 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   // variant that kept them live spilled registers and ran 2 % slower)
   const int qb = a.causal ? (a.num_qblocks - 1 - (int)(a.grouped ? blockIdx.y : blockIdx.x)) : (int)blockIdx.x;
   const int bh = a.grouped ? (int)(blockIdx.z * gridDim.x + blockIdx.x) : (int)blockIdx.y;
-  const int n_ktiles = a.Npad / 128;
+  const int n_ktiles = a.Npad_k / 128;
   int nt[kNQ];
   int T = 0;
 #pragma unroll
   for (int q = 0; q < kNQ; ++q) {
     const int qt = kNQ * qb + q;
-    nt[q] = qt >= n_ktiles ? 0 : (a.causal ? qt + 1 : n_ktiles);
+    // causal: up to the key tile of the last visible key of the tile's last real row
+    nt[q] = qt * 128 >= a.N ? 0 : (a.causal ? min(n_ktiles, (min(qt * 128 + 127, a.N - 1) + a.koff) / 128 + 1)
+                                            : n_ktiles);
     T = max(T, nt[q]);
   }
 
@@ -189,6 +208,8 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       mbar_arrive_expect_tx(q_full, qbytes);
       for (int q = 0; q < kNQ; ++q)
         if (nt[q] > 0) tma_load_3d(smem + L::off_q + q * L::kQ, &tm_q, q_full, 0, (kNQ * qb + q) * 128, bh);
+      // the key/value slice of this query head
+      const int bkv = kv_slice(a, bh);
       int issued_k = 0, issued_v = 0;
       for (int j = 0; j < T; ++j) {
         const int s = j % kStages, n = j / kStages;
@@ -197,14 +218,14 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(&k_full[s], L::kK);
-        tma_load_5d(smem + L::off_k + s * L::kK, &tm_k, &k_full[s], 0, 0, 0, j, bh);
+        tma_load_5d(smem + L::off_k + s * L::kK, &tm_k, &k_full[s], 0, 0, 0, j, bkv);
         issued_k = j + 1;
         if (j >= kStages && !mbar_wait(&v_empty[s], (n - 1) & 1, abort_flag)) {
           fail(abort_flag, a.err, kErrProducer);
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kV);
-        tma_load_4d(smem + L::off_v + s * L::kV, &tm_v, &v_full[s], j * 128, 0, 0, bh);
+        tma_load_4d(smem + L::off_v + s * L::kV, &tm_v, &v_full[s], j * 128, 0, 0, bkv);
         issued_v = j + 1;
       }
       // Drain: every load issued into shared memory must land before exit.
@@ -306,8 +327,8 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       const uint32_t t_o = tmem + lane_off + kColO + q * D;
       const uint32_t t_h = tmem + lane_off + kColH;
       uint8_t* prow0 = smem + L::off_p + 2 * q * L::kP + r * 128;  // buffer 0; buffer 1 is kP further
-      const float* ksc = a.k_scale + (size_t)bh * (a.Npad / 64);
-      const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad + h * 64 : nullptr;
+      const float* ksc = a.k_scale + (size_t)kv_slice(a, bh) * (a.Npad_k / 64);
+      const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad_k + h * 64 : nullptr;
       // m: running row max of the logits (log2 units); l: this half's running
       // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
@@ -344,9 +365,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         const int kbase = j * 128 + h * 64;
         // visible keys of this row among the half's 64 form the prefix c < lim
         int lim = 64;
-        if (kbase + 63 >= a.N || (a.causal && j == qt)) {
-          lim = min(lim, a.N - kbase);
-          if (a.causal) lim = min(lim, row - kbase + 1);
+        if (kbase + 63 >= a.Nk || (a.causal && kbase + 63 > row + a.koff)) {
+          lim = min(lim, a.Nk - kbase);
+          if (a.causal) lim = min(lim, row + a.koff - kbase + 1);
         }
         // FP16 mode: the tile's 64 bias values, loaded before the wait for S
         // hides their latency; the FP32 mode, whose 576 threads leave no
@@ -508,8 +529,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       } else {
         tc_fence_after();
         const float inv_l = __fdiv_rn(1.0f, l);
-        const float* vs = a.v_scale + (size_t)bh * D + h * kHalfD;
-        OutT* orow = (OutT*)a.out + ((size_t)bh * a.N + row) * D + h * kHalfD;
+        const int bh_e = query_slice(a);
+        const float* vs = a.v_scale + (size_t)kv_slice(a, bh_e) * D + h * kHalfD;
+        OutT* orow = (OutT*)a.out + ((size_t)bh_e * a.N + row) * D + h * kHalfD;
 #pragma unroll 1
         for (int i = 0; i < D / 64; ++i) {
           // o[e] = channel h d/2 + 32 i + e of this row
@@ -637,14 +659,14 @@ static bool make_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mq, CUten
 
 // The attention kernel's K and V^T tiles in pair order: shared-memory row
 // 2i + e holds key 64e + i of the 128-key tile (K), channel (d/2) e + i (V^T).
-//   K   [BH][Npad][d]: dims (d, e = 2, i = 64, tile, bh), box (d, 2, 64, 1, 1)
-//   V^T [BH][d][Npad]: dims (Npad, e = 2, i = d/2, bh), box (128, 2, d/2, 1)
+//   K   [BHkv][Npk][d]: dims (d, e = 2, i = 64, tile, bh), box (d, 2, 64, 1, 1)
+//   V^T [BHkv][d][Npk]: dims (Npk, e = 2, i = d/2, bh), box (128, 2, d/2, 1)
 static bool make_pair_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mk, CUtensorMap* mv) {
-  const uint64_t D = (uint64_t)pb.d, Np = (uint64_t)pb.Npad;
-  const uint64_t kd[5] = {D, 2, 64, Np / 128, (uint64_t)pb.BH};
+  const uint64_t D = (uint64_t)pb.d, Np = (uint64_t)pb.npk();
+  const uint64_t kd[5] = {D, 2, 64, Np / 128, (uint64_t)pb.bh_kv()};
   const uint64_t ks[4] = {64 * D, D, 128 * D, Np * D};
   const uint32_t kb[5] = {(uint32_t)D, 2, 64, 1, 1};
-  const uint64_t vd[4] = {Np, 2, D / 2, (uint64_t)pb.BH};
+  const uint64_t vd[4] = {Np, 2, D / 2, (uint64_t)pb.bh_kv()};
   const uint64_t vs[3] = {(D / 2) * Np, Np, D * Np};
   const uint32_t vb[4] = {128, 2, (uint32_t)(D / 2), 1};
   return make_tmap_u8_nd(mk, w.k_codes, 5, kd, ks, kb, (int)D) && make_tmap_u8_nd(mv, w.vt_codes, 4, vd, vs, vb, 128);
@@ -659,15 +681,16 @@ static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const 
   // be shared by host threads and devices
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
   if (e != cudaSuccess) return e;
-  const int G = causal_slice_group(BH, 2.0 * a.Npad * D, 80e6);
+  const int G = causal_slice_group(BH, 2.0 * a.Npad_k * D, 80e6);
   const dim3 grid = a.grouped ? dim3(G, a.num_qblocks, BH / G) : dim3(a.num_qblocks, BH);
   kern<<<grid, Roles<F16ACC>::kThreads, L::alloc, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mk_rows;
-  if (!make_maps(w, pb, &mq, &mk_rows) || !make_pair_maps(w, pb, &mk, &mv)) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv;
+  if (!make_tmap_u8_3d(&mq, w.q_codes, pb.d, pb.Npad, pb.BH, pb.d, 128) || !make_pair_maps(w, pb, &mk, &mv))
+    return cudaErrorInvalidValue;
   AttnArgs a;
   a.q_scale = w.q_scale;
   a.k_scale = w.k_scale;
@@ -677,6 +700,11 @@ cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, floa
   a.err = w.error;
   a.N = pb.N;
   a.Npad = pb.Npad;
+  a.Nk = pb.nk();
+  a.Npad_k = pb.npk();
+  a.koff = pb.nk() - pb.N;
+  a.Hq = pb.hq();
+  a.G = pb.G;
   a.causal = pb.causal;
   const bool f16 = pb.mode == 1;
   const int nq = f16 ? 1 : 2;

@@ -84,7 +84,14 @@ struct QuantArgs {
   int* err;
   int BH, N, Npad, smooth_q, n_items;
   float Vr;
+  // tensors this pass handles: kRolesQ, kRolesKV or both (the per-head
+  // problem: Q, K and V share heads and tokens).  With grouped key/value heads
+  // the K/V pass writes the Q-smoothing bias of the G query heads of each
+  // key/value slice, reading their means from q_mean_g.
+  int roles, G;
+  const float* q_mean_g;
 };
+constexpr int kRolesQ = 1, kRolesKV = 2;
 
 // Shared-memory image of one 64-token tile of a [.., D] 16-bit tensor as TMA
 // writes it with SWIZZLE_128B: D/64 boxes of 64 rows x 128 bytes, the 16-byte
@@ -238,7 +245,8 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    const bool need_q = PASS == kCodesPass || a.smooth_q || FP4;
+    const bool do_q = (a.roles & kRolesQ) != 0, do_kv = (a.roles & kRolesKV) != 0;
+    const bool need_q = do_q && (PASS == kCodesPass || a.smooth_q || FP4);
     for (int it = 0;; ++it) {
       const int b = it & 1;
       // the codes pass walks the items backwards: the slices the statistics
@@ -257,26 +265,27 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
       }
       const int bh = item / nb, blk = item % nb;
       info[b] = make_int4(item, bh, blk, 0);
-      uint32_t bytes = (uint32_t)L::kTile * (need_q ? 3 : 2);
-      if (PASS == kCodesPass) bytes += FP4 ? (uint32_t)(D * 4) * (a.smooth_q ? 2 : 1) + 16u
-                                           : (uint32_t)(D * 4) * (a.smooth_q ? 3 : 2);
+      uint32_t bytes = (uint32_t)L::kTile * ((need_q ? 1 : 0) + (do_kv ? 2 : 0));
+      if (PASS == kCodesPass)
+        bytes += FP4 ? (uint32_t)(D * 4) * (a.smooth_q ? 2 : 1) + 16u
+                     : (uint32_t)(D * 4) * ((do_kv ? 2 : 0) + (do_q && a.smooth_q ? 1 : 0));
       mbar_arrive_expect_tx(&full[b], bytes);
       uint8_t* dst = sm + b * L::kItem;
 #pragma unroll
       for (int x = 0; x < D / 64; ++x) {
         const int off = x * kTok * kBoxBytes;
-        tma_load_3d(dst + off, &tm_k, &full[b], x * kBoxBytes, blk * kTok, bh);
+        if (do_kv) tma_load_3d(dst + off, &tm_k, &full[b], x * kBoxBytes, blk * kTok, bh);
         if (need_q) tma_load_3d(dst + L::kTile + off, &tm_q, &full[b], x * kBoxBytes, blk * kTok, bh);
-        tma_load_3d(dst + 2 * L::kTile + off, &tm_v, &full[b], x * kBoxBytes, blk * kTok, bh);
+        if (do_kv) tma_load_3d(dst + 2 * L::kTile + off, &tm_v, &full[b], x * kBoxBytes, blk * kTok, bh);
       }
       if (PASS == kCodesPass) {
         // the slice's means and V multipliers (written by the fold kernel)
         float* sl = reinterpret_cast<float*>(sm + L::kTiles) + b * (3 * D);
-        bulk_load(sl, a.k_mean + (size_t)bh * D, D * 4, &full[b]);
-        if (a.smooth_q) bulk_load(sl + D, a.q_mean + (size_t)bh * D, D * 4, &full[b]);
+        if (do_kv || FP4) bulk_load(sl, a.k_mean + (size_t)bh * D, D * 4, &full[b]);
+        if (a.smooth_q && (do_q || FP4)) bulk_load(sl + D, a.q_mean + (size_t)bh * D, D * 4, &full[b]);
         if (FP4)
           bulk_load(sl + 2 * D, a.gscale + (size_t)bh * 4, 16, &full[b]);
-        else
+        else if (do_kv)
           bulk_load(sl + 2 * D, a.v_mul + (size_t)bh * D, D * 4, &full[b]);
       }
     }
@@ -350,7 +359,8 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
       // order; W <= u < 2W: the same for Q (smooth_q); 2W <= u < 3W: |V|
       // maxima of word u - 2W (exact max / min of the raw values).
       const int role = tid / W, word = tid % W;
-      if (role < 3 && (role != 1 || a.smooth_q)) {
+      const bool mine = role == 1 ? (a.roles & kRolesQ) && a.smooth_q : (a.roles & kRolesKV) != 0;
+      if (role < 3 && mine) {
         uint32_t o[8];
         col_offsets(word, 0, o);
         float* p = a.part + role * plane + ((size_t)bh * nchunks + blk) * D + 2 * word;
@@ -531,6 +541,7 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
         const int cw = tid % W, r0 = (tid / W) * RPG;  // this thread's column word and first row
         uint32_t o[8];
         col_offsets(cw, r0, o);
+        const bool do_q = (a.roles & kRolesQ) != 0, do_kv = (a.roles & kRolesKV) != 0;
         // A: per (row group, word) max and min of the raw K and Q values
         {
           uint32_t kx = P::kNegInf, kn = P::kPosInf, qx = P::kNegInf, qn = P::kPosInf;
@@ -538,12 +549,16 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
           for (int r = 0; r < RPG; ++r) {
             if (rows == kTok || r0 + r < rows) {
               const uint32_t off = o[r & 7] + 1024 * (r >> 3);
-              const uint32_t uk = lds<uint32_t>(sb + tk + off);
-              const uint32_t uq = lds<uint32_t>(sb + tq + off);
-              kx = P::max(kx, uk);
-              kn = P::min(kn, uk);
-              qx = P::max(qx, uq);
-              qn = P::min(qn, uq);
+              if (do_kv) {
+                const uint32_t uk = lds<uint32_t>(sb + tk + off);
+                kx = P::max(kx, uk);
+                kn = P::min(kn, uk);
+              }
+              if (do_q) {
+                const uint32_t uq = lds<uint32_t>(sb + tq + off);
+                qx = P::max(qx, uq);
+                qn = P::min(qn, uq);
+              }
             }
           }
           mm[0][tid] = make_uint2(kx, kn);
@@ -563,7 +578,7 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
             n = P::min(n, e.y);
           }
           float am = 0.f;
-          if ((isk ? rows : rows - 32 * g) > 0) {
+          if ((isk ? do_kv : do_q) && (isk ? rows : rows - 32 * g) > 0) {
             float x0, x1, n0, n1;
             unpack2<T>(x, x0, x1);
             unpack2<T>(n, n0, n1);
@@ -592,8 +607,8 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
           mq0 = fmaxf(mq0, red[WPG + i]);
           mq1 = fmaxf(mq1, red[2 * WPG + i]);
         }
-        if (tid == 0) a.k_scale[(size_t)bh * (a.Npad / 64) + t0 / 64] = mk > 0.f ? __fdiv_rn(mk, 127.0f) : 0.f;
-        if (tid == 1 || tid == 2) {
+        if (tid == 0 && do_kv) a.k_scale[(size_t)bh * (a.Npad / 64) + t0 / 64] = mk > 0.f ? __fdiv_rn(mk, 127.0f) : 0.f;
+        if ((tid == 1 || tid == 2) && do_q) {
           const float m = tid == 1 ? mq0 : mq1;
           a.q_scale[(size_t)bh * (a.Npad / 32) + t0 / 32 + (tid - 1)] = m > 0.f ? __fdiv_rn(m, 127.0f) : 0.f;
         }
@@ -611,6 +626,7 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
 #pragma unroll 1
           for (int which = 0; which < 2; ++which) {
             const bool isk = which == 0;
+            if (!(isk ? do_kv : do_q)) continue;
             const bool sub = isk || a.smooth_q;
             const uint32_t src = isk ? tk : tq;
             const uint32_t mean = isk ? kmean : qmean;
@@ -650,7 +666,7 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
             }
           }
         }
-        if (a.smooth_q && tid < kTok) {
+        if (a.smooth_q && do_kv && tid < kTok && do_q) {
           // Q-smoothing bias of token t0 + tid: fma chain over channels of
           // mean_q[c] * k~[c] in channel order (k~ recomputed from the tile)
           const int row = tid;
@@ -671,8 +687,34 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
             }
           }
           a.q_bias[(size_t)bh * a.Npad + t0 + row] = acc;
+        } else if (a.smooth_q && do_kv && tid < kTok) {
+          // K/V pass with its own query heads: the bias of each of the G query
+          // heads of this key/value slice (query slice bh * G + g), the same
+          // chain with that head's mean read from global memory
+          const int row = tid;
+#pragma unroll 1
+          for (int g = 0; g < a.G; ++g) {
+            const float* mq = a.q_mean_g + ((size_t)bh * a.G + g) * D;
+            float acc = 0.f;
+            if (row < rows) {
+#pragma unroll 1
+              for (int c0 = 0; c0 < D; c0 += 8) {
+                const uint4 v4 = lds<uint4>(sb + tk + swz(row, 2 * c0));
+                const uint32_t uu[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  float lo, hi;
+                  unpack2<T>(uu[j], lo, hi);
+                  const int c = c0 + 2 * j;
+                  acc = __fmaf_rn(__ldg(mq + c), __fsub_rn(lo, lds<float>(kmean + 4 * c)), acc);
+                  acc = __fmaf_rn(__ldg(mq + c + 1), __fsub_rn(hi, lds<float>(kmean + 4 * c + 4)), acc);
+                }
+              }
+            }
+            a.q_bias[((size_t)bh * a.G + g) * a.Npad + t0 + row] = acc;
+          }
         }
-        {
+        if (do_kv) {
           // V: thread = word cw (channels 2cw, 2cw+1) x rows r0 .. r0+RPG-1;
           // e4m3 codes of v * (Vr / absmax_c), written transposed [c][t]
           const float mul0 = lds<float>(vmul + 8 * cw), mul1 = lds<float>(vmul + 8 * cw + 4);
@@ -775,7 +817,8 @@ __global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
   __shared__ __align__(8) uint64_t bar[2];
   __shared__ int abort_s;
   const int bh = blockIdx.x, c = threadIdx.x;
-  const int which = blockIdx.y == 0 ? 0 : blockIdx.y == 1 ? 2 : 1;  // part plane
+  // part plane: K sums, V maxima, Q sums (a Q-only pass folds Q sums alone)
+  const int which = a.roles == kRolesQ ? 1 : blockIdx.y == 0 ? 0 : blockIdx.y == 1 ? 2 : 1;
   const int nchunks = a.Npad / 64;
   const int nvalid = (a.N + 63) / 64;
   if (c == 0) {
@@ -924,6 +967,9 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
   a.smooth_q = pb.smooth_q;
   a.Vr = Vr;
   a.n_items = pb.BH * (pb.Npad / kTok);
+  a.roles = kRolesQ | kRolesKV;
+  a.G = 1;
+  a.q_mean_g = w.q_mean;
 
   // 16-bit [BH][N][D] inputs seen as bytes: rows of 2D bytes, boxes of
   // 128 bytes x 64 tokens (rows past N read as zero)
@@ -961,7 +1007,103 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
                        tv, a);
 }
 
+// Grouped key/value heads and / or separate query and key lengths (INT8/FP8
+// modes): the same kernels in two passes, one over Q's slices and tokens and
+// one over K/V's.  Order: Q statistics and fold (Q smoothing only), K/V
+// statistics and fold, K/V codes (with the bias of every query head of each
+// key/value slice, which needs the Q means), Q codes.  Every launch after the
+// first is programmatic and waits for its predecessor, so each sees all
+// earlier results.
+template <typename T, int D>
+cudaError_t quant_run_split(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
+                            const WsPtrs& w, cudaStream_t s) {
+  const int BHq = pb.BH, BHkv = pb.bh_kv(), Npq = pb.Npad, Npk = pb.npk();
+  const size_t plane_q = (size_t)BHq * (Npq / 64) * D, plane_kv = (size_t)BHkv * (Npk / 64) * D;
+  QuantArgs a;
+  a.q_codes = w.q_codes;
+  a.k_codes = w.k_codes;
+  a.vt_codes = w.vt_codes;
+  a.q_scale = w.q_scale;
+  a.k_scale = w.k_scale;
+  a.v_scale = w.v_scale;
+  a.k_mean = w.k_mean;
+  a.q_mean = w.q_mean;
+  a.q_bias = w.q_bias;
+  a.gscale = w.global_scale;
+  a.err = w.error;
+  a.smooth_q = pb.smooth_q;
+  a.Vr = Vr;
+  a.G = pb.G;
+  a.q_mean_g = w.q_mean;
+  QuantArgs aq = a, akv = a;
+  aq.roles = kRolesQ;
+  aq.BH = BHq;
+  aq.N = pb.N;
+  aq.Npad = Npq;
+  aq.n_items = BHq * (Npq / kTok);
+  aq.part = w.scratch;  // Q sums in plane 1 of two
+  aq.v_mul = nullptr;
+  akv.roles = kRolesKV;
+  akv.BH = BHkv;
+  akv.N = pb.nk();
+  akv.Npad = Npk;
+  akv.n_items = BHkv * (Npk / kTok);
+  akv.part = w.scratch + 2 * plane_q;  // K sums plane 0, V maxima plane 2
+  akv.v_mul = akv.part + 3 * plane_kv;
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t row_bytes = (uint64_t)D * 2;
+  if (!make_tmap_u8_3d(&tq, q, row_bytes, pb.N, BHq, kBoxBytes, kTok) ||
+      !make_tmap_u8_3d(&tk, k, row_bytes, pb.nk(), BHkv, kBoxBytes, kTok) ||
+      !make_tmap_u8_3d(&tv, v, row_bytes, pb.nk(), BHkv, kBoxBytes, kTok))
+    return cudaErrorInvalidValue;
+  const size_t smem = QLayout<D>::kBytes + 1024;
+  LaunchFacts f0, f1;
+  cudaError_t e = launch_facts<T, D, kStatsPass, false>(smem, &f0);
+  if (e != cudaSuccess) return e;
+  e = launch_facts<T, D, kCodesPass, false>(smem, &f1);
+  if (e != cudaSuccess) return e;
+  auto grid = [](const QuantArgs& x, const LaunchFacts& f) {
+    return dim3((unsigned)fmin((double)x.n_items, (double)f.sms * f.per_sm));
+  };
+  bool pdl = false;  // the first launch follows the caller's work normally
+  if (pb.smooth_q) {
+    e = launch_kernel(quant_pass_kernel<T, D, kStatsPass, false>, grid(aq, f0), dim3(kThreadsQ), smem, s, pdl, tq,
+                      tq, tq, aq);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(quant_fold_kernel<D>, dim3(BHq, 1), dim3(D), 0, s, true, aq);
+    if (e != cudaSuccess) return e;
+    pdl = true;
+  }
+  e = launch_kernel(quant_pass_kernel<T, D, kStatsPass, false>, grid(akv, f0), dim3(kThreadsQ), smem, s, pdl, tk, tk,
+                    tv, akv);
+  if (e != cudaSuccess) return e;
+  e = launch_kernel(quant_fold_kernel<D>, dim3(BHkv, 2), dim3(D), 0, s, true, akv);
+  if (e != cudaSuccess) return e;
+  e = launch_kernel(quant_pass_kernel<T, D, kCodesPass, false>, grid(akv, f1), dim3(kThreadsQ), smem, s, true, tk, tk,
+                    tv, akv);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(quant_pass_kernel<T, D, kCodesPass, false>, grid(aq, f1), dim3(kThreadsQ), smem, s, true, tq,
+                       tq, tq, aq);
+}
+
 }  // namespace
+
+// Scratch floats of the two-pass quantization with grouped key/value heads or
+// separate lengths: Q partials (two planes), K/V partials (three planes), V
+// multipliers.
+size_t quant_scratch_floats_split(int BHq, int Npq, int BHkv, int Npk, int d) {
+  return (size_t)2 * BHq * (Npq / 64) * d + (size_t)3 * BHkv * (Npk / 64) * d + (size_t)BHkv * d;
+}
+
+cudaError_t launch_quant_split(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
+                               const WsPtrs& w, cudaStream_t s) {
+  if (pb.dtype == 0)
+    return pb.d == 128 ? quant_run_split<__half, 128>(q, k, v, pb, Vr, w, s)
+                       : quant_run_split<__half, 64>(q, k, v, pb, Vr, w, s);
+  return pb.d == 128 ? quant_run_split<__nv_bfloat16, 128>(q, k, v, pb, Vr, w, s)
+                     : quant_run_split<__nv_bfloat16, 64>(q, k, v, pb, Vr, w, s);
+}
 
 // Scratch floats the quantization pass needs (chunk partials, V multipliers).
 size_t quant_scratch_floats(int BH, int Npad, int d, int mode) {

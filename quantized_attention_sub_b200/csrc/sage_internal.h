@@ -25,8 +25,16 @@ struct WsPtrs {
   float* scratch;  // statistics partials, then the per-channel V multipliers
 };
 
+// BH = B * Hq query slices of N query rows (padded to Npad); with grouped
+// key/value heads (G = Hq / Hkv > 1) and / or a key length Nk != N the last
+// fields describe the keys; 0 there means "the same as the queries".
 struct Problem {
   int BH, N, Npad, d, dtype, smooth_q, mode, causal;
+  int Hq = 0, G = 1, Nk = 0, Npad_k = 0;
+  int nk() const { return Nk ? Nk : N; }
+  int npk() const { return Npad_k ? Npad_k : Npad; }
+  int bh_kv() const { return BH / G; }
+  int hq() const { return Hq ? Hq : 1; }
 };
 
 // Causal attention grids run (G, query blocks, B*H/G): the CTAs of G slices
@@ -64,6 +72,12 @@ inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, 
 // [BH][d].  NVFP4: partials [7][BH][Npad/64][d] (the same three planes, then
 // K maxima, K minima, Q maxima, Q minima of the raw values).
 size_t quant_scratch_floats(int BH, int Npad, int d, int mode);
+
+// The same with grouped key/value heads or separate query and key lengths
+// (INT8/FP8 modes): separate passes over Q and over K/V.
+size_t quant_scratch_floats_split(int BHq, int Npq, int BHkv, int Npk, int d);
+cudaError_t launch_quant_split(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
+                               const WsPtrs& w, cudaStream_t s);
 
 // Smoothing statistics + INT8 Q/K + FP8 V (+ bias), enqueued on `s`.
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,

@@ -76,3 +76,30 @@ def test_bad_pointers_rejected_before_any_launch(lib):
     # debug tile out of range
     st = lib.sage_debug_qk_s32(vp(4096), ws_bytes, 1, 2, 128, 64, 0, 1, 0, vp(4096), vp(0))
     assert st == api.SAGE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 6, 4, 128, 128, 64, 0), api.SAGE_ERR_INVALID_ARG),      # Hq not a multiple of Hkv
+    ((1, 8, 2, 128, 128, 128, 2), api.SAGE_ERR_UNSUPPORTED),     # NVFP4 with grouped heads
+    ((1, 8, 0, 128, 128, 64, 0), api.SAGE_ERR_INVALID_ARG),
+    ((1, 8, 2, 128, 0, 64, 0), api.SAGE_ERR_INVALID_ARG),
+])
+def test_gqa_shapes_rejected_on_host(lib, args, status):
+    out = api.WsLayout()
+    assert lib.sage_workspace_layout_gqa(*args, ctypes.byref(out)) == status
+
+
+def test_gqa_layout_reduces_to_per_head_layout(lib):
+    for (B, H, N, d, mode) in [(1, 4, 1000, 128, 0), (2, 3, 257, 64, 1), (1, 2, 512, 128, 2)]:
+        a, b = api.sage_workspace_layout(B, H, N, d, mode), api.sage_workspace_layout_gqa(B, H, H, N, N, d, mode)
+        assert all(getattr(a, f) == getattr(b, f) for f, _ in api.WsLayout._fields_)
+    L = api.sage_workspace_layout_gqa(2, 8, 2, 100, 3000, 128, 0)
+    assert L.k_codes - L.q_codes >= 2 * 8 * 128 * 128 and L.vt_codes - L.k_codes >= 2 * 2 * 3072 * 128
+
+
+def test_gqa_causal_needs_nq_le_nk(lib):
+    vp = ctypes.c_void_p
+    ws = api.sage_workspace_layout_gqa(1, 4, 2, 300, 200, 64, 0).total
+    st = lib.sage_attn_fwd_gqa(vp(4096), vp(4096), vp(4096), vp(4096), 1, 4, 2, 300, 200, 64, 1, 0, 0, 0, vp(4096), ws,
+                               vp(0))
+    assert st == api.SAGE_ERR_UNSUPPORTED
