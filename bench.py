@@ -133,12 +133,12 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle timing (the reported baseline and the reference arm)
 # --------------------------------------------------------------------------
-def oracle_sample(w, max_rows, threads=0):
+def oracle_sample(w, max_rows, threads=0, keep=None):
     """The CPU oracle as it stands on a bounded sample of the workload: slice
     (b=0, h=0) quantized in full, attention for `max_rows` evenly spaced
     query rows.  Returns (ops of the sampled rows at 4*d per key the row sees
     -- all N keys, or i+1 for row i under a causal mask; seconds; threads;
-    rows)."""
+    rows).  keep: a dict that receives the inputs, rows and oracle output."""
     import oracle as orc
     if threads:
         orc.set_num_threads(threads)
@@ -148,13 +148,28 @@ def oracle_sample(w, max_rows, threads=0):
     t0 = time.perf_counter()
     if w.mode == 2:
         qz = orc.quantize_nvfp4(f(q), f(k), f(v), smooth_q=w.smooth_q)
-        orc.attention_nvfp4(qz, w.causal, rows=rows)
+        o = orc.attention_nvfp4(qz, w.causal, rows=rows)
     else:
         qz = orc.quantize_int8_fp8(f(q), f(k), f(v), smooth_q=w.smooth_q, mode=w.mode)
-        orc.attention_int8_fp8(qz, w.causal, rows=rows)
+        o = orc.attention_int8_fp8(qz, w.causal, rows=rows)
     dt = time.perf_counter() - t0
+    if keep is not None:
+        keep.update(q=q, k=k, v=v, rows=rows, out=o)
     keys = (rows.astype(np.float64) + 1.0).sum() if w.causal else float(w.N) * len(rows)
     return float(4.0 * w.d * keys), dt, orc.num_threads(), len(rows)
+
+
+def gpu_vs_oracle(w, keep, dev):
+    """The GPU path (sage_attn_fwd) on the oracle sample's slice: max-abs and
+    relative L1 of its output against the oracle's, both in the output dtype."""
+    q, k, v = [keep[n].to(dev) for n in ("q", "k", "v")]
+    out = api.attn_fwd(q, k, v, causal=w.causal, mode=w.mode, smooth_q=w.smooth_q)
+    torch.cuda.synchronize()
+    got = out.float().cpu().reshape(w.N, w.d).numpy()[keep["rows"]].astype(np.float64)
+    ref = torch.from_numpy(keep["out"][0]).to(inputs.DTYPES[w.dtype]).double().numpy()
+    diff = np.abs(got - ref)
+    return {"max_abs": float(diff.max()), "rel_l1": float(diff.sum() / np.abs(ref).sum()),
+            "sample": "slice (b0,h0) of the CPU sample, %d rows" % len(keep["rows"])}
 
 
 def run_reference(args, w, ws, rank):
@@ -321,27 +336,31 @@ def summarize(w, t, probe, hbm):
     return s
 
 
+def accuracy_metrics(o_test, o_ref) -> dict:
+    """Cosine similarity, relative L1 and RMSE of O' against O (the metrics of
+    the SageAttention2++ summary, App. A.2)."""
+    a = np.asarray(o_test, np.float64).ravel()
+    b = np.asarray(o_ref, np.float64).ravel()
+    return {"cos": float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b))),
+            "rel_l1": float(np.abs(a - b).sum() / np.abs(b).sum()),
+            "rmse": float(np.sqrt(np.mean((a - b) ** 2)))}
+
+
 def accuracy_leg(w, t, rows_n=48):
-    """cos / rel-L1 / RMSE of the GPU output against fp64 attention of the
-    unquantized inputs, and max-abs / rel-L1 against the CPU oracle, on
-    `rows_n` sampled query rows of slice (b0, h0)."""
-    import oracle as orc
+    """cos / rel-L1 / RMSE of the GPU output against softmax(Q K^T / sqrt(d)) V
+    of the unquantized inputs, computed in float64 (torch, on the device), on
+    `rows_n` evenly spaced query rows of slice (b0, h0)."""
     B, H, N, d = w.shape()
-    f = lambda x: x.reshape(B * H, N, d)[:1].float().cpu().numpy()
-    q, k, v = f(t["q"]), f(t["k"]), f(t["v"])
-    rows = np.unique(np.linspace(0, N - 1, rows_n).astype(np.int32))
-    got = t["out"].reshape(B * H, N, d)[:1, rows].float().cpu().numpy()
-    ref64 = orc.attention_fp64(q, k, v, w.causal, rows=rows)
-    if w.mode == 2:
-        o32 = orc.attention_nvfp4(orc.quantize_nvfp4(q, k, v, smooth_q=w.smooth_q), w.causal, rows=rows)
-    else:
-        o32 = orc.attention_int8_fp8(orc.quantize_int8_fp8(q, k, v, smooth_q=w.smooth_q, mode=w.mode), w.causal,
-                                     rows=rows)
-    o_ref = torch.from_numpy(o32).to(inputs.DTYPES[w.dtype]).float().numpy()
-    diff = np.abs(got.astype(np.float64) - o_ref)
-    return {"vs_fp64": orc.accuracy(got, ref64), "vs_oracle": {
-        "max_abs": float(diff.max()), "rel_l1": float(diff.sum() / np.abs(o_ref).sum())},
-        "sample": "slice (b0,h0), %d evenly spaced query rows" % len(rows)}
+    sl = lambda x: x.reshape(B * H, N, d)[0].double()
+    q, k, v = sl(t["q"]), sl(t["k"]), sl(t["v"])
+    rows = torch.from_numpy(np.unique(np.linspace(0, N - 1, rows_n).astype(np.int64))).to(q.device)
+    s = (q[rows] @ k.T) / np.sqrt(d)
+    if w.causal:
+        s = s.masked_fill(torch.arange(N, device=q.device)[None, :] > rows[:, None], float("-inf"))
+    ref = torch.softmax(s, dim=1) @ v
+    got = t["out"].reshape(B * H, N, d)[0, rows].double()
+    return {"vs_fp64": accuracy_metrics(got.cpu().numpy(), ref.cpu().numpy()),
+            "sample": "slice (b0,h0), %d evenly spaced query rows" % len(rows)}
 
 
 def e2e_leg(w, t, dev, steps, ws):
@@ -401,6 +420,32 @@ def e2e_leg(w, t, dev, steps, ws):
     return {"value": inputs.attention_ops(w) * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": e2e_ms,
             "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
             "pipelined": "step i+1's H2D copy overlaps step i's compute and step i-1's D2H copy"}
+
+
+def fused_leg(w, dev, steps, warmup):
+    """The whole step through sage_attn_fwd_fused (Q quantized inside the
+    attention kernel) against the same step through sage_attn_fwd, CUDA
+    events on the launch stream; device-resident inputs."""
+    B, H, N, d = w.shape()
+    dcode = api.DTYPE_CODE[inputs.DTYPES[w.dtype]]
+    q, k, v = [t.to(dev) for t in inputs.generate(w, device="cuda")]
+    out = torch.empty_like(q)
+    wsbuf = api.alloc_workspace(B, H, N, d, w.mode, dev)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, fn in (("unfused", api.sage_attn_fwd), ("fused", api.sage_attn_fwd_fused)):
+        for _ in range(warmup):
+            fn(q, k, v, out, B, H, N, d, w.causal, w.mode, dcode, w.smooth_q, wsbuf, wsbuf.numel(), stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn(q, k, v, out, B, H, N, d, w.causal, w.mode, dcode, w.smooth_q, wsbuf, wsbuf.numel(), stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[name + "_ms"] = e0.elapsed_time(e1) / steps
+    api.sage_check(wsbuf, wsbuf.numel(), stream)
+    res["value_fused"] = inputs.attention_ops(w) / (res["fused_ms"] * 1e-3) / 1e12
+    return res
 
 
 def per_config_leg(dev, steps, probe, hbm, skip):
@@ -498,6 +543,12 @@ def main():
     torch.cuda.empty_cache()
 
     per_config = per_config_leg(dev, min(args.steps, 10), probe, hbm, w.name) if extras else None
+    fused = None
+    if extras and w.mode != 2:
+        fused = {w.name: fused_leg(w, dev, min(args.steps, 10), 3)}
+        torch.cuda.empty_cache()
+        fused["llm_prefill"] = fused_leg(workload("llm_prefill"), dev, 10, 3)
+        torch.cuda.empty_cache()
 
     line = {"metric": METRIC, "value": value,
             "unit": "TOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -517,10 +568,16 @@ def main():
         line["accuracy"] = acc
     if per_config is not None:
         line["per_config"] = per_config
+    if fused is not None:
+        # Q quantized inside the attention kernel (sage_attn_fwd_fused), whole step
+        line["fused_q"] = fused
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle as orc
         orc.build()
-        ops, dt, thr, nr = oracle_sample(w, 2048)
+        keep = {}
+        ops, dt, thr, nr = oracle_sample(w, 2048, keep=keep)
+        if "accuracy" in line:
+            line["accuracy"]["vs_oracle"] = gpu_vs_oracle(w, keep, dev)
         cpu = {"value": ops / dt / 1e12, "unit": "TOPS", "cores": thr, "kind": "oracle",
                "sample": "slice (b0,h0) quantized in full + attention of %d evenly spaced query rows; %.1f s "
                          "(ops counted over the keys each row sees)" % (nr, dt)}

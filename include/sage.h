@@ -163,6 +163,21 @@ SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, 
                           int causal, int mode, int dtype, int smooth_q, void* ws, size_t ws_bytes,
                           sage_stream_t stream);
 
+/* sage_attn_fwd with Q quantized inside the attention kernel: each CTA
+ * loads its 128-row tiles of the caller's 16-bit Q and quantizes them itself
+ * (the per-block Q quantization of the SageAttention2++ summary, Sec. 2.1,
+ * fused into the FlashAttention-style kernel of Sec. 2) with the steps of
+ * sage_quantize_qkv, so Q makes one trip from HBM instead of three (read,
+ * codes written, codes read).  K and V are quantized beforehand (with
+ * smooth_q, Q's means and the bias too).  The output is bit-identical to
+ * sage_attn_fwd's; the workspace (sage_workspace_size bytes) afterwards holds
+ * the K/V codes, scales, means and bias but not Q's codes or scales.
+ * INT8/FP8 modes (SAGE_MODE_NVFP4 returns SAGE_ERR_UNSUPPORTED); other
+ * arguments as for sage_attn_fwd; out must be 16-byte aligned. */
+SAGE_API sage_status sage_attn_fwd_fused(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                                         int d, int causal, int mode, int dtype, int smooth_q, void* ws,
+                                         size_t ws_bytes, sage_stream_t stream);
+
 /* sage_attn_fwd with the P~ and V quantization ranges chosen by the caller:
  * P~ = e4m3(p * Pr), V codes e4m3(v * Vr / absmax), O rescaled by 1 / Pr.
  * The SageAttention2++ summary (Sec. 3.1) narrows both so that an FP16

@@ -21,7 +21,7 @@ DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
 
 EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_quantize_qkv_static",
             "sage_attn_quantized",
-            "sage_attn_fwd", "sage_attn_fwd_ranges", "sage_workspace_layout_gqa", "sage_quantize_qkv_gqa",
+            "sage_attn_fwd", "sage_attn_fwd_fused", "sage_attn_fwd_ranges", "sage_workspace_layout_gqa", "sage_quantize_qkv_gqa",
             "sage_attn_quantized_gqa", "sage_attn_fwd_gqa", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_probe_mma_rate",
             "sage_check", "sage_last_error")
 PROBE_I8, PROBE_F8_F32ACC, PROBE_F8_F16ACC, PROBE_BF16, PROBE_FP4 = range(5)
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.sage_attn_quantized.restype = i
         L.sage_attn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.sage_attn_fwd.restype = i
+        L.sage_attn_fwd_fused.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_attn_fwd_fused.restype = i
         f = ctypes.c_float
         L.sage_attn_fwd_ranges.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, vp, sz, vp]
         L.sage_attn_fwd_ranges.restype = i
@@ -136,6 +138,11 @@ def sage_attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, 
 def sage_attn_fwd(q, k, v, out, B, H, N, d, causal, mode, dtype, smooth_q, ws, ws_bytes, stream=None):
     _raise(lib().sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, int(causal), mode, dtype,
                                int(smooth_q), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def sage_attn_fwd_fused(q, k, v, out, B, H, N, d, causal, mode, dtype, smooth_q, ws, ws_bytes, stream=None):
+    _raise(lib().sage_attn_fwd_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, int(causal), mode, dtype,
+                                     int(smooth_q), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def sage_attn_fwd_ranges(q, k, v, out, B, H, N, d, causal, mode, dtype, smooth_q, Pr, Vr, ws, ws_bytes,

@@ -334,6 +334,30 @@ sage_status sage_attn_fwd_ranges(const void* q, const void* k, const void* v, vo
   return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, smooth_q, mode, Pr, stream, true);
 }
 
+sage_status sage_attn_fwd_fused(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int d,
+                                int causal, int mode, int dtype, int smooth_q, void* ws, size_t ws_bytes,
+                                sage_stream_t stream) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (mode == SAGE_MODE_NVFP4)
+    return set_err(SAGE_ERR_UNSUPPORTED, "the fused forward covers the INT8/FP8 modes%s");
+  if (!q || !k || !v || !out) return set_err(SAGE_ERR_INVALID_ARG, "null input or output pointer%s");
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
+  if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v) | ((uintptr_t)out)) % 16)
+    return set_err(SAGE_ERR_INVALID_ARG, "inputs and output must be 16-byte aligned%s");
+  const sage_ws_layout L = layout_of(B, H, N, d, mode);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != SAGE_OK) return st;
+  sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
+  if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
+    return st;
+  const sage::WsPtrs w = resolve(ws, L);
+  if ((st = cuda_status(sage::launch_quant_split(q, k, v, pb, default_vr(mode), w, (cudaStream_t)stream, true),
+                        "quantize launch")) != SAGE_OK)
+    return st;
+  return cuda_status(sage::launch_attn_i8f8_fused_q(w, q, out, pb, default_pr(mode), (cudaStream_t)stream),
+                     "attention launch");
+}
+
 sage_status sage_workspace_layout_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode, sage_ws_layout* out) {
   sage_status st = check_shape_gqa(B, Hq, Hkv, Nq, Nk, d, mode);
   if (st != SAGE_OK) return st;

@@ -42,6 +42,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "sage_internal.h"
 #include "sage_ptx.cuh"
 #include "sage_softmax.cuh"
@@ -75,7 +77,8 @@ struct Smem {
   static constexpr int off_v = off_k + kStages * kK;
   static constexpr int off_p = off_v + kStages * kV;  // [query tile NQ][buffer 2]
   static constexpr int off_bar = off_p + 2 * NQ * kP;
-  static constexpr int bytes = off_bar + 256;
+  static constexpr int off_qmx = off_bar + 256;  // fused Q: granule maxima [query tile 2][granule 4][warp 2]
+  static constexpr int bytes = off_bar + 512;
   static constexpr int alloc = bytes + 1024;  // room to align the base to 1024
 };
 
@@ -84,6 +87,7 @@ struct AttnArgs {
   const float* k_scale;
   const float* v_scale;
   const float* bias;  // null unless smooth_q
+  const float* q_mean;  // fused Q with smooth_q: the per-channel Q means
   void* out;
   int* err;
   int N, Npad, causal, num_qblocks;     // query rows (padded), causal flag, CTAs per slice
@@ -121,7 +125,7 @@ SAGE_DEV int kv_slice(const AttnArgs& a, int bh) {
 
 }  // namespace
 
-template <int D, typename OutT, bool HAS_BIAS, bool F16ACC>
+template <int D, typename OutT, bool HAS_BIAS, bool F16ACC, bool FUSED_Q>
 __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -146,7 +150,8 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   uint64_t* p_full = s_full + 4;              // [2]
   uint64_t* o_done = s_full + 6;              // [2]
   uint64_t* mma_fin = s_full + 8;
-  uint32_t* tmem_slot = (uint32_t*)(s_full + 9);
+  uint64_t* q_ready = s_full + 9;             // [2] fused Q: the tile's codes are in place
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 11);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,6 +188,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       mbar_init(&s_free[q], 8);   // 8 softmax warps per query tile
       mbar_init(&p_full[q], 8);
       mbar_init(&o_done[q], 1);
+      mbar_init(&q_ready[q], 8);
     }
     mbar_init(mma_fin, 1);
     *abort_flag = 0;
@@ -204,10 +210,21 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       uint32_t qbytes = 0;
-      for (int q = 0; q < kNQ; ++q) qbytes += nt[q] > 0 ? L::kQ : 0;
+      for (int q = 0; q < kNQ; ++q) qbytes += nt[q] > 0 ? (FUSED_Q ? 2 * L::kQ : L::kQ) : 0;
       mbar_arrive_expect_tx(q_full, qbytes);
-      for (int q = 0; q < kNQ; ++q)
-        if (nt[q] > 0) tma_load_3d(smem + L::off_q + q * L::kQ, &tm_q, q_full, 0, (kNQ * qb + q) * 128, bh);
+      for (int q = 0; q < kNQ; ++q) {
+        if (nt[q] == 0) continue;
+        if (FUSED_Q) {
+          // the raw 16-bit Q tile, 128 rows x 2d bytes, into this query tile's P~
+          // buffers (free until its first P~): boxes of 128 bytes x 128 rows, 128B swizzle
+#pragma unroll
+          for (int x = 0; x < 2 * D / 128; ++x)
+            tma_load_3d(smem + L::off_p + 2 * q * L::kP + x * 128 * 128, &tm_q, q_full, x * 128, (kNQ * qb + q) * 128,
+                        bh);
+        } else {
+          tma_load_3d(smem + L::off_q + q * L::kQ, &tm_q, q_full, 0, (kNQ * qb + q) * 128, bh);
+        }
+      }
       // the key/value slice of this query head
       const int bkv = kv_slice(a, bh);
       int issued_k = 0, issued_v = 0;
@@ -244,7 +261,14 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       constexpr uint32_t idesc_pv = idesc_make(F16ACC ? 0u : 1u, 0u, 0u, 128, D);
       const uint32_t q_base = smem_u32(smem + L::off_q), k_base = smem_u32(smem + L::off_k);
       const uint32_t v_base = smem_u32(smem + L::off_v), p_base = smem_u32(smem + L::off_p);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+      bool ok = true;
+      if (FUSED_Q) {
+        // the softmax warps quantize the Q tiles
+        for (int q = 0; q < kNQ && ok; ++q)
+          if (nt[q] > 0) ok = mbar_wait(&q_ready[q], 0, abort_flag);
+      } else {
+        ok = mbar_wait(q_full, 0, abort_flag);
+      }
       auto issue_s = [&](int q, int j) {
         const uint32_t qa = q_base + q * L::kQ, kb = k_base + (j % kStages) * L::kK;
 #pragma unroll
@@ -320,7 +344,84 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
     if (nt[q] > 0) {
       const int qt = kNQ * qb + q;
       const int row = qt * 128 + r;
-      const float sq = a.q_scale[(size_t)bh * (a.Npad / 32) + (row >> 5)];
+      float sq;
+      bool ok = true;
+      if (!FUSED_Q) {
+        sq = a.q_scale[(size_t)bh * (a.Npad / 32) + (row >> 5)];
+      } else {
+        // Q quantized here (SageAttention2++ summary Sec. 2.1: per-block Q
+        // scales), with the steps of the quantization pass: x~ = x - mean_q
+        // (smooth_q), granule of 32 rows: a = max |x~| over valid rows, scale
+        // a / 127, code = rint_even(x~ * (127 / a)); rows past N give 0.
+        ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
+        float x[kHalfD];
+        float am = 0.f;
+        if (ok) {
+          const uint8_t* raw = smem + L::off_p + 2 * q * L::kP;
+#pragma unroll
+          for (int k = 0; k < kHalfD / 8; ++k) {
+            // 16-byte chunk k of this half row: byte b = 2 (d/2) h + 16 k of the row
+            const int b = h * D + 16 * k;
+            const uint4 u = *reinterpret_cast<const uint4*>(raw + (b >> 7) * (128 * 128) + r * 128 +
+                                                            ((((b >> 4) & 7) ^ (r & 7)) << 4));
+            const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float lo, hi;
+              if constexpr (sizeof(OutT) == 2 && std::is_same<OutT, __half>::value) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&uu[e]));
+                lo = f.x;
+                hi = f.y;
+              } else {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
+                lo = f.x;
+                hi = f.y;
+              }
+              x[8 * k + 2 * e] = lo;
+              x[8 * k + 2 * e + 1] = hi;
+            }
+          }
+          if (HAS_BIAS) {
+            const float* mq = a.q_mean + (size_t)bh * D + h * kHalfD;
+#pragma unroll
+            for (int c = 0; c < kHalfD; ++c) x[c] = __fsub_rn(x[c], __ldg(mq + c));
+          }
+          if (row < a.N) {
+#pragma unroll
+            for (int c = 0; c < kHalfD; ++c) am = fmaxf(am, fabsf(x[c]));
+          }
+        }
+        // granule maximum: this warp's 16 rows, then the other warp of the granule
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        float* qmx = (float*)(smem + L::off_qmx) + q * 8 + (wq & 3) * 2;
+        if (lane == 0) qmx[wq >> 2] = am;
+        named_bar_sync(1 + q * 4 + (wq & 3), 64);
+        const float ag = fmaxf(qmx[0], qmx[1]);
+        sq = ag > 0.f ? __fdiv_rn(ag, 127.0f) : 0.f;
+        const float inv = ag > 0.f ? __fdiv_rn(127.0f, ag) : 0.f;
+        // codes into the Q operand tile (K-major, d-byte rows in the d-byte swizzle)
+        uint8_t* qrow = smem + L::off_q + q * L::kQ + r * D;
+#pragma unroll
+        for (int k = 0; k < kHalfD / 16; ++k) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float z[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) z[i] = __fadd_rn(__fmul_rn(x[16 * k + 4 * e + i], inv), 12582912.0f);
+            const uint32_t lo = __byte_perm(__float_as_uint(z[0]), __float_as_uint(z[1]), 0x0040);
+            const uint32_t hi = __byte_perm(__float_as_uint(z[2]), __float_as_uint(z[3]), 0x0040);
+            w4[e] = row < a.N ? __byte_perm(lo, hi, 0x5410) : 0u;
+          }
+          const int c = (D / 32) * h + k;  // 16-byte chunk of the code row
+          const int sw = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+          *reinterpret_cast<uint4*>(qrow + (sw << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_ready[q]);
+      }
       // S columns [0, 128) of this query tile (two loads of 64), O columns of this
       // tile, H_0 (H_1 is D columns further)
       const uint32_t t_s = tmem + lane_off + q * 128;
@@ -333,7 +434,6 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
       float alpha_prev = 0.f;  // FP16 accumulator: rescale factor of the tile whose partials are pending
-      bool ok = true;
       // FP16 accumulator, after P~V(jt) completed: acc = (alpha_jt * acc + h_0) + h_1
       // over this thread's O columns (the first tile starts from acc = 0).
       auto fold_partials = [&](int jt, float alpha_t) {
@@ -359,7 +459,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       };
       // K scales of both 64-key granules of the tile, loaded one tile ahead
       float2 ks_next = *reinterpret_cast<const float2*>(ksc);
-      for (int j = 0; j < nt[q]; ++j) {
+      for (int j = 0; ok && j < nt[q]; ++j) {
         const float2 ks = ks_next;
         if (j + 1 < nt[q]) ks_next = *reinterpret_cast<const float2*>(ksc + 2 * (j + 1));
         const int kbase = j * 128 + h * 64;
@@ -672,10 +772,10 @@ static bool make_pair_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mk, 
   return make_tmap_u8_nd(mk, w.k_codes, 5, kd, ks, kb, (int)D) && make_tmap_u8_nd(mv, w.vt_codes, 4, vd, vs, vb, 128);
 }
 
-template <int D, typename OutT, bool HAS_BIAS, bool F16ACC>
+template <int D, typename OutT, bool HAS_BIAS, bool F16ACC, bool FUSED_Q>
 static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                             int BH, cudaStream_t s) {
-  auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS, F16ACC>;
+  auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS, F16ACC, FUSED_Q>;
   using L = Smem<D, Roles<F16ACC>::kNQ>;
   // set on every launch: the attribute is per device, and a cached flag would
   // be shared by host threads and devices
@@ -687,15 +787,21 @@ static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const 
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s) {
+// q_raw: null, or the caller's 16-bit Q [BH, N, d] for the fused variant
+// (then mq maps it as bytes: rows of 2d bytes, boxes of 128 bytes x 128 rows).
+static cudaError_t launch_attn(const WsPtrs& w, const void* q_raw, void* out, const Problem& pb, float Pr,
+                               cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  if (!make_tmap_u8_3d(&mq, w.q_codes, pb.d, pb.Npad, pb.BH, pb.d, 128) || !make_pair_maps(w, pb, &mk, &mv))
-    return cudaErrorInvalidValue;
+  const bool fused = q_raw != nullptr;
+  const bool qmap = fused ? make_tmap_u8_3d(&mq, q_raw, 2 * (uint64_t)pb.d, pb.N, pb.BH, 128, 128)
+                          : make_tmap_u8_3d(&mq, w.q_codes, pb.d, pb.Npad, pb.BH, pb.d, 128);
+  if (!qmap || !make_pair_maps(w, pb, &mk, &mv)) return cudaErrorInvalidValue;
   AttnArgs a;
   a.q_scale = w.q_scale;
   a.k_scale = w.k_scale;
   a.v_scale = w.v_scale;
   a.bias = pb.smooth_q ? w.q_bias : nullptr;
+  a.q_mean = w.q_mean;
   a.out = out;
   a.err = w.error;
   a.N = pb.N;
@@ -718,14 +824,25 @@ cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, floa
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)pb.d));
   a.log2Pr = (float)log2((double)Pr);
   const bool bias = a.bias != nullptr;
-#define SAGE_RUN(DD, TT, BB, FF) run_attn<DD, TT, BB, FF>(mq, mk, mv, a, pb.BH, s)
-#define SAGE_RUN_F(DD, TT, BB) (f16 ? SAGE_RUN(DD, TT, BB, true) : SAGE_RUN(DD, TT, BB, false))
+#define SAGE_RUN(DD, TT, BB, FF, QQ) run_attn<DD, TT, BB, FF, QQ>(mq, mk, mv, a, pb.BH, s)
+#define SAGE_RUN_Q(DD, TT, BB, FF) (fused ? SAGE_RUN(DD, TT, BB, FF, true) : SAGE_RUN(DD, TT, BB, FF, false))
+#define SAGE_RUN_F(DD, TT, BB) (f16 ? SAGE_RUN_Q(DD, TT, BB, true) : SAGE_RUN_Q(DD, TT, BB, false))
 #define SAGE_RUN_B(DD, TT) (bias ? SAGE_RUN_F(DD, TT, true) : SAGE_RUN_F(DD, TT, false))
   if (pb.d == 128) return pb.dtype == 0 ? SAGE_RUN_B(128, __half) : SAGE_RUN_B(128, __nv_bfloat16);
   return pb.dtype == 0 ? SAGE_RUN_B(64, __half) : SAGE_RUN_B(64, __nv_bfloat16);
 #undef SAGE_RUN_B
 #undef SAGE_RUN_F
+#undef SAGE_RUN_Q
 #undef SAGE_RUN
+}
+
+cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s) {
+  return launch_attn(w, nullptr, out, pb, Pr, s);
+}
+
+cudaError_t launch_attn_i8f8_fused_q(const WsPtrs& w, const void* q_raw, void* out, const Problem& pb, float Pr,
+                                     cudaStream_t s) {
+  return launch_attn(w, q_raw, out, pb, Pr, s);
 }
 
 cudaError_t launch_timeout_probe(const WsPtrs& w, cudaStream_t s) {

@@ -1014,11 +1014,16 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
 // key/value slice, which needs the Q means), Q codes.  Every launch after the
 // first is programmatic and waits for its predecessor, so each sees all
 // earlier results.
+// skip_q_codes: leave Q's codes and scales to the attention kernel, which
+// quantizes each Q tile itself (the fused forward); only Q's statistics run.
+// With equal shapes the two passes share the per-head layout's three
+// partial planes (K sums 0, Q sums 1, V maxima 2).
 template <typename T, int D>
 cudaError_t quant_run_split(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
-                            const WsPtrs& w, cudaStream_t s) {
+                            const WsPtrs& w, cudaStream_t s, bool skip_q_codes) {
   const int BHq = pb.BH, BHkv = pb.bh_kv(), Npq = pb.Npad, Npk = pb.npk();
   const size_t plane_q = (size_t)BHq * (Npq / 64) * D, plane_kv = (size_t)BHkv * (Npk / 64) * D;
+  const bool shared_planes = BHq == BHkv && Npq == Npk;
   QuantArgs a;
   a.q_codes = w.q_codes;
   a.k_codes = w.k_codes;
@@ -1048,7 +1053,7 @@ cudaError_t quant_run_split(const void* q, const void* k, const void* v, const P
   akv.N = pb.nk();
   akv.Npad = Npk;
   akv.n_items = BHkv * (Npk / kTok);
-  akv.part = w.scratch + 2 * plane_q;  // K sums plane 0, V maxima plane 2
+  akv.part = shared_planes ? w.scratch : w.scratch + 2 * plane_q;  // K sums plane 0, V maxima plane 2
   akv.v_mul = akv.part + 3 * plane_kv;
 
   CUtensorMap tq, tk, tv;
@@ -1082,7 +1087,7 @@ cudaError_t quant_run_split(const void* q, const void* k, const void* v, const P
   if (e != cudaSuccess) return e;
   e = launch_kernel(quant_pass_kernel<T, D, kCodesPass, false>, grid(akv, f1), dim3(kThreadsQ), smem, s, true, tk, tk,
                     tv, akv);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || skip_q_codes) return e;
   return launch_kernel(quant_pass_kernel<T, D, kCodesPass, false>, grid(aq, f1), dim3(kThreadsQ), smem, s, true, tq,
                        tq, tq, aq);
 }
@@ -1097,12 +1102,12 @@ size_t quant_scratch_floats_split(int BHq, int Npq, int BHkv, int Npk, int d) {
 }
 
 cudaError_t launch_quant_split(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
-                               const WsPtrs& w, cudaStream_t s) {
+                               const WsPtrs& w, cudaStream_t s, bool skip_q_codes) {
   if (pb.dtype == 0)
-    return pb.d == 128 ? quant_run_split<__half, 128>(q, k, v, pb, Vr, w, s)
-                       : quant_run_split<__half, 64>(q, k, v, pb, Vr, w, s);
-  return pb.d == 128 ? quant_run_split<__nv_bfloat16, 128>(q, k, v, pb, Vr, w, s)
-                     : quant_run_split<__nv_bfloat16, 64>(q, k, v, pb, Vr, w, s);
+    return pb.d == 128 ? quant_run_split<__half, 128>(q, k, v, pb, Vr, w, s, skip_q_codes)
+                       : quant_run_split<__half, 64>(q, k, v, pb, Vr, w, s, skip_q_codes);
+  return pb.d == 128 ? quant_run_split<__nv_bfloat16, 128>(q, k, v, pb, Vr, w, s, skip_q_codes)
+                     : quant_run_split<__nv_bfloat16, 64>(q, k, v, pb, Vr, w, s, skip_q_codes);
 }
 
 // Scratch floats the quantization pass needs (chunk partials, V multipliers).

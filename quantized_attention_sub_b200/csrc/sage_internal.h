@@ -76,8 +76,10 @@ size_t quant_scratch_floats(int BH, int Npad, int d, int mode);
 // The same with grouped key/value heads or separate query and key lengths
 // (INT8/FP8 modes): separate passes over Q and over K/V.
 size_t quant_scratch_floats_split(int BHq, int Npq, int BHkv, int Npk, int d);
+// skip_q_codes: Q statistics only (the fused forward quantizes Q in the
+// attention kernel); with equal shapes the per-head layout's scratch serves.
 cudaError_t launch_quant_split(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
-                               const WsPtrs& w, cudaStream_t s);
+                               const WsPtrs& w, cudaStream_t s, bool skip_q_codes = false);
 
 // Smoothing statistics + INT8 Q/K + FP8 V (+ bias), enqueued on `s`.
 cudaError_t launch_quant_int8_fp8(const void* q, const void* k, const void* v, const Problem& pb, float Vr,
@@ -92,6 +94,10 @@ size_t static_scratch_floats();
 // Fused attention (FP32 or FP16 PV accumulator).  Launched normally: a
 // programmatic launch behind the codes pass measured slower on video_dit.
 cudaError_t launch_attn_i8f8(const WsPtrs& w, void* out, const Problem& pb, float Pr, cudaStream_t s);
+// The same with Q quantized inside the attention kernel from the caller's
+// 16-bit Q ([BH, N, d]); the workspace holds K/V codes, scales, means, bias.
+cudaError_t launch_attn_i8f8_fused_q(const WsPtrs& w, const void* q_raw, void* out, const Problem& pb, float Pr,
+                                     cudaStream_t s);
 
 // Fused NVFP4 attention (kind::mxf4nvf4 for S and P~V, FP32 accumulator); d = 128.
 cudaError_t launch_attn_fp4(const WsPtrs& w, void* out, const Problem& pb, cudaStream_t s);
