@@ -56,8 +56,9 @@ HEADLINE = "sweep_N32768_d128_full"
 # DRAM bytes (read + write) of one attention launch of the headline workload:
 # one ncu capture of the kernel as it stands on B4 H32 N8192 d128 (inputs
 # above L2), scaled by the token count (non-causal attention traffic is the
-# codes read once plus the output, linear in N).  None until captured.
-TRAFFIC_BYTES = {}
+# codes read once plus the output, linear in N): 403,055,360 B read +
+# 232,906,752 B written at N = 8192, times 4.
+TRAFFIC_BYTES = {"sweep_N32768_d128_full": 4 * (403055360 + 232906752)}
 
 MODE_NAMES = ["INT8_FP8", "INT8_FP8_F16ACC", "NVFP4"]
 MODE_INFO = {
