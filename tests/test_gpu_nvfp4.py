@@ -106,6 +106,16 @@ def test_nvfp4_quantize_bitexact(N, d, dtype, law, smooth_q):
     assert_fp4_bitexact(g, oracle_fp4(q, k, v, smooth_q), d, smooth_q)
 
 
+def test_nvfp4_quantize_many_slices_bitexact():
+    """B1 H40 N2048 d128 with Q smoothing: codes, block scales, global
+    scales, means and bias of many slices equal the oracle's."""
+    w = inputs.variant(inputs.WORKLOADS["unit"], N=2048, d=128, H=40, dtype="bf16", law="student_t3",
+                       smooth_q=True, mode=api.MODE_NVFP4, seed=7400)
+    q, k, v = [t.cuda() for t in inputs.generate(w)]
+    _, g = run_quant_fp4(q, k, v, True)
+    assert_fp4_bitexact(g, oracle_fp4(q, k, v, True), 128, True)
+
+
 def test_nvfp4_quantize_edge_values():
     """A zero V channel, an all-zero Q slice (global scale 0), a constant K
     block, a value far above the rest (subnormal block scales elsewhere)."""

@@ -71,6 +71,16 @@ def test_quantize_bitexact(N, d, dtype, law, smooth_q, mode):
     assert_quant_bitexact(g, oracle_quant(qkv, mode, smooth_q), smooth_q)
 
 
+@pytest.mark.parametrize("H,N,d,smooth_q", [(40, 2048, 128, False), (80, 2048, 64, True)])
+def test_quantize_many_slices_bitexact(H, N, d, smooth_q):
+    """Many slices (40 and 80, more than the persistent passes' CTAs can
+    take in one round of chunks): every code, scale, mean and bias equals
+    the oracle's."""
+    w = small_workload(N, d, "fp16", "qk_bias" if smooth_q else "k_bias", smooth_q, 0, H=H)
+    qkv, ws, g = run_quant(w, 0, smooth_q)
+    assert_quant_bitexact(g, oracle_quant(qkv, 0, smooth_q), smooth_q)
+
+
 def test_quantize_edge_values():
     """Zero channels, constant tokens, a zero granule, huge and tiny values."""
     w = small_workload(200, 64, "fp16", "k_bias", True, 0)
