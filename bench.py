@@ -433,18 +433,25 @@ def fused_leg(w, dev, steps, warmup):
     out = torch.empty_like(q)
     wsbuf = api.alloc_workspace(B, H, N, d, w.mode, dev)
     stream = torch.cuda.current_stream()
-    res = {}
-    for name, fn in (("unfused", api.sage_attn_fwd), ("fused", api.sage_attn_fwd_fused)):
+    fns = (("unfused", api.sage_attn_fwd), ("fused", api.sage_attn_fwd_fused))
+    for _, fn in fns:
         for _ in range(warmup):
             fn(q, k, v, out, B, H, N, d, w.causal, w.mode, dcode, w.smooth_q, wsbuf, wsbuf.numel(), stream)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            fn(q, k, v, out, B, H, N, d, w.causal, w.mode, dcode, w.smooth_q, wsbuf, wsbuf.numel(), stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        res[name + "_ms"] = e0.elapsed_time(e1) / steps
+    # the two calls alternate (three rounds, median of each), so that clock
+    # drift under the power cap falls on both alike
+    times = {name: [] for name, _ in fns}
+    for _ in range(3):
+        for name, fn in fns:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn(q, k, v, out, B, H, N, d, w.causal, w.mode, dcode, w.smooth_q, wsbuf, wsbuf.numel(), stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times[name].append(e0.elapsed_time(e1) / steps)
     api.sage_check(wsbuf, wsbuf.numel(), stream)
+    res = {name + "_ms": float(np.median(t)) for name, t in times.items()}
+    res["rounds"] = "3 alternating rounds of %d steps each, medians" % steps
     res["value_fused"] = inputs.attention_ops(w) / (res["fused_ms"] * 1e-3) / 1e12
     return res
 

@@ -173,7 +173,9 @@ SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, 
  * sage_attn_fwd's; the workspace (sage_workspace_size bytes) afterwards holds
  * the K/V codes, scales, means and bias but not Q's codes or scales.
  * INT8/FP8 modes (SAGE_MODE_NVFP4 returns SAGE_ERR_UNSUPPORTED); other
- * arguments as for sage_attn_fwd; out must be 16-byte aligned. */
+ * arguments as for sage_attn_fwd; out must be 16-byte aligned.  Speed: the
+ * saved Q traffic is offset by each CTA quantizing its Q tiles before its
+ * first MMA, so on a B200 the call runs at about the speed of sage_attn_fwd. */
 SAGE_API sage_status sage_attn_fwd_fused(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
                                          int d, int causal, int mode, int dtype, int smooth_q, void* ws,
                                          size_t ws_bytes, sage_stream_t stream);

@@ -111,6 +111,22 @@ def test_qk_s32_tiles_bitexact(N, d):
             assert np.array_equal(out.cpu().numpy(), ref), (bh, qt, kt)
 
 
+@pytest.mark.parametrize("N,d", [(32768, 128), (8192, 64)])
+def test_qk_s32_tiles_bitexact_long(N, d):
+    """One slice at the sweep's token counts (the headline N = 32768, d = 128):
+    INT32 S tiles across the whole key range -- first, last, diagonal and
+    off-diagonal -- equal the oracle's integer products."""
+    w = inputs.variant(inputs.sweep(N, d, False), B=1, H=1)
+    qkv, ws, g = run_quant(w, 0, False)
+    T = N // 128
+    out = torch.empty(128, 128, dtype=torch.int32, device="cuda")
+    for qt, kt in [(0, 0), (T - 1, T - 1), (0, T - 1), (T - 1, 0), (T // 2, T // 3), (T // 3, 2 * T // 3)]:
+        api.sage_debug_qk_s32(ws, ws.numel(), 1, 1, N, d, 0, qt, kt, out)
+        api.sage_check(ws, ws.numel())
+        ref = orc.qk_s32(g["q_codes"][0, qt * 128:(qt + 1) * 128], g["k_codes"][0, kt * 128:(kt + 1) * 128])
+        assert np.array_equal(out.cpu().numpy(), ref), (qt, kt)
+
+
 ATTN_SMALL = [
     # (N, d, dtype, law, smooth_q, causal, mode)
     (128, 64, "fp16", "k_bias", False, False, 0),
