@@ -232,6 +232,36 @@ def test_full_size_video_dit_sampled_rows():
     compare_out(got, ref32, flip, "fp16", "video_dit")
 
 
+def test_max_size_sampled_slices():
+    """The largest problem the C ABI accepts in element count: B1 H16383
+    N1024 d128, B*H*Npad*d = 2^31 - 2^17 (the limit is < 2^31), 16383
+    slices in the attention grid.  Inputs drawn on the GPU (12.9 GB), the
+    whole problem quantized and attended; three slices spread over the index
+    range are checked: codes and scales bit-exact, the output on sampled
+    rows within the parity bounds (so no index past 2^31 bytes wraps)."""
+    w = inputs.variant(inputs.sweep(1024, 128, False), B=1, H=16383)
+    B, H, N, d = w.shape()
+    assert B * H * N * d < (1 << 31) <= B * (H + 1) * N * d  # one more slice is refused
+    q, k, v = inputs.generate(w, device="cuda")
+    ws = api.alloc_workspace(B, H, N, d, 0)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd(q, k, v, out, B, H, N, d, False, 0, 0, False, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    views = api.ws_views(ws, B, H, N, d, 0)
+    rows = np.array([0, 1, 127, 128, 511, 512, 1022, 1023], np.int32)
+    for bh in (0, H // 2, H - 1):
+        sl = lambda t: t[:, bh:bh + 1].contiguous()
+        oz = oracle_quant((sl(q), sl(k), sl(v)), 0, False)
+        g = {n: views[n][bh:bh + 1].cpu().numpy() for n in ("q_codes", "k_codes", "vt_codes", "q_scale", "k_scale",
+                                                              "v_scale", "k_mean")}
+        assert_quant_bitexact(g, oz, False)
+        ref32, flip = orc.attention_int8_fp8(oz, False, rows=rows, with_flip=True)
+        got = out[0, bh].float().cpu().numpy()[rows][None]
+        compare_out(got, ref32, flip, "fp16", "max size, slice %d" % bh)
+    del q, k, v, ws, out
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("N,d,causal", [(8192, 128, False), (2048, 64, True), (8192, 64, True), (16384, 64, True),
                                          (4096, 128, True), (16384, 128, True), (1024, 64, False)])
 def test_sweep_points_sampled_rows(N, d, causal):
