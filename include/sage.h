@@ -21,8 +21,8 @@
  *     stream.  The library never allocates, frees or synchronizes, except
  *     sage_check, which synchronizes the given stream.
  *   - All work is enqueued asynchronously on `stream` (0 = legacy default).
- *   - Supported: d in {64, 128}, N >= 1, B*H >= 1, B*H*Npad*d < 2^31 where
- *     Npad = ceil(N / 128) * 128.  Other values return SAGE_ERR_UNSUPPORTED
+ *   - Supported: d in {64, 128}, N >= 1, 1 <= B*H <= 65535, B*H*Npad*d < 2^31
+ *     where Npad = ceil(N / 128) * 128.  Other values return SAGE_ERR_UNSUPPORTED
  *     or SAGE_ERR_INVALID_ARG before any launch; a launch failure returns
  *     SAGE_ERR_CUDA.  sage_last_error() gives a message for the last non-OK
  *     status of the calling thread.
