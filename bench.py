@@ -509,7 +509,9 @@ def main():
     hbm = peaks["hbm_gbs"]
     extras = ws == 1 and not args.no_extras
 
-    probe = probe_peaks(dev, sm_count) if extras else None
+    # every rank probes its own GPU (no collective), so the roofline fraction
+    # has the same denominator at every N
+    probe = probe_peaks(dev, sm_count) if not args.no_extras else None
 
     clocks = ClockSampler(local)
     t = time_workload(w, dev, args.steps, args.warmup, seed_rank=rank, clocks=clocks, ws=ws)
