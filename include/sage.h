@@ -175,8 +175,8 @@ SAGE_API sage_status sage_attn_fwd(const void* q, const void* k, const void* v, 
  * INT8/FP8 modes (SAGE_MODE_NVFP4 returns SAGE_ERR_UNSUPPORTED); other
  * arguments as for sage_attn_fwd; out must be 16-byte aligned.  Speed: the
  * saved Q traffic is largely offset by each CTA quantizing its Q tiles before
- * its first MMA: on a B200 the call is 0.3 % faster than sage_attn_fwd at
- * B4 H32 N32768 d128 and 2 % slower at B1 H32 N8192 d128 causal. */
+ * its first MMA: on a B200 the call runs within 0.3 % of sage_attn_fwd at
+ * B4 H32 N32768 d128 and 2-3 % slower at B1 H32 N8192 d128 causal. */
 SAGE_API sage_status sage_attn_fwd_fused(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
                                          int d, int causal, int mode, int dtype, int smooth_q, void* ws,
                                          size_t ws_bytes, sage_stream_t stream);
