@@ -287,6 +287,67 @@ def attention_int8_fp8(qz: dict, causal: bool, rows=None, with_flip: bool = Fals
     return (out, flip) if with_flip else out
 
 
+Q_BLOCK = 128  # query rows per smoothing block (the attention's query tile)
+
+
+def quantize_int8_fp8_blocksmooth(q, k, v, mode: int, Vr: float | None = None) -> dict:
+    """Preprocessing with Q smoothed per block of 128 query rows instead of
+    per slice (the pages say only that Q is smoothed, SageAttention2
+    abstract): block b's mean is the channel mean of its valid rows (the
+    per-slice mean's fixed order applied to the block), its rows are
+    quantized in their 32-row granules after subtracting that mean, and its
+    bias row is the per-slice bias formula with that mean, over every key.
+    K, V and their statistics as in quantize_int8_fp8.  Returns the same
+    dict with q_mean [BH, nblk, d] and q_bias [BH, nblk, Npad]."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BH, N, d = q.shape
+    Np = npad(N)
+    nblk = Np // Q_BLOCK
+    if Vr is None:
+        Vr = VR_F16ACC if mode == MODE_INT8_FP8_F16ACC else VR_FP32ACC
+    mean_k = channel_mean(k)
+    amax_v = channel_absmax(v)
+    kc, sk = quant_int8(k, mean_k, K_GRANULE)
+    vt, sv = quant_v_fp8(v, amax_v, Vr)
+    qc = np.zeros((BH, Np, d), np.int8)
+    sq = np.zeros((BH, Np // Q_GRANULE), np.float32)
+    mean_q = np.empty((BH, nblk, d), np.float32)
+    bias = np.empty((BH, nblk, Np), np.float32)
+    for b in range(nblk):
+        r0, r1 = b * Q_BLOCK, min(N, (b + 1) * Q_BLOCK)
+        xb = np.ascontiguousarray(q[:, r0:r1])
+        mb = channel_mean(xb)
+        cb, sb = quant_int8(xb, mb, Q_GRANULE)
+        qc[:, r0:r0 + Q_BLOCK] = cb
+        sq[:, r0 // Q_GRANULE:(r0 + Q_BLOCK) // Q_GRANULE] = sb
+        mean_q[:, b] = mb
+        bias[:, b] = q_bias(k, mean_k, mb)
+    return dict(q_codes=qc, q_scale=sq, k_codes=kc, k_scale=sk, vt_codes=vt, v_scale=sv,
+                k_mean=mean_k, q_mean=mean_q, q_bias=bias, v_absmax=amax_v,
+                N=N, d=d, mode=mode)
+
+
+def attention_int8_fp8_blocksmooth(qz: dict, causal: bool, rows=None, with_flip: bool = False):
+    """attention_int8_fp8 on quantize_int8_fp8_blocksmooth's output: each
+    query row takes the bias row of its 128-row block.  Runs the per-slice
+    attention once per block on that block's rows with that block's bias."""
+    N, d = qz["N"], qz["d"]
+    BH = qz["q_codes"].shape[0]
+    all_rows = np.arange(N, dtype=np.int32) if rows is None else np.asarray(rows, np.int32)
+    out = np.empty((BH, len(all_rows), d), np.float32)
+    flip = np.empty((BH, len(all_rows), d), np.float32) if with_flip else None
+    blocks = all_rows // Q_BLOCK
+    for b in np.unique(blocks):
+        sel = np.nonzero(blocks == b)[0]
+        view = dict(qz, q_bias=np.ascontiguousarray(qz["q_bias"][:, b]))
+        res = attention_int8_fp8(view, causal, rows=all_rows[sel], with_flip=with_flip)
+        if with_flip:
+            out[:, sel], flip[:, sel] = res
+        else:
+            out[:, sel] = res
+    return (out, flip) if with_flip else out
+
+
 def quantize_int8_fp8_gqa(q, k, v, smooth_q: bool, mode: int, Vr: float | None = None) -> dict:
     """Preprocessing with grouped key/value heads and separate lengths: q
     [B, Hq, Nq, d], k and v [B, Hkv, Nk, d].  Each tensor is smoothed and
