@@ -199,9 +199,9 @@ def run_reference(args, w, ws, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, ws):
+def config_of(w, ws, q_blocks=False):
     return {"workload": w.name, "B": w.B * ws, "H": w.H, "N": w.N, "d": w.d, "dtype": w.dtype,
-            "causal": w.causal, "mode": MODE_NAMES[w.mode], "smooth_q": w.smooth_q,
+            "causal": w.causal, "mode": MODE_NAMES[w.mode], "smooth_q": w.smooth_q, "q_blocks": q_blocks,
             "parallelism": "replicas x%d (independent (b,h) slices per rank)" % ws,
             "l2": "inputs (3 x %.0f MB) larger than the 126 MB L2; no flush" % (
                 w.B * w.H * w.N * w.d * 2 / 1e6)}
@@ -267,24 +267,31 @@ def mode_peak(mode, probe, which="burst"):
 # --------------------------------------------------------------------------
 # Device timing of one workload
 # --------------------------------------------------------------------------
-def time_workload(w, dev, steps, warmup, seed_rank=0, clocks=None, ws=1):
+def time_workload(w, dev, steps, warmup, seed_rank=0, clocks=None, ws=1, q_blocks=False):
     """Quantize + attention steps on device-resident inputs; CUDA events on
     the launch stream around each kernel group.  Returns the timings and the
-    tensors (for the accuracy and e2e legs)."""
+    tensors (for the accuracy and e2e legs).  q_blocks: Q smoothed per
+    128-row block (the sage_*_blocksmooth calls)."""
     B, H, N, d = w.shape()
     dcode = api.DTYPE_CODE[inputs.DTYPES[w.dtype]]
     wr = inputs.variant(w, seed=replicas.rank_seed(w.seed, seed_rank))
     q, k, v = [t.to(dev) for t in inputs.generate(wr, device="cuda")]
     out = torch.empty_like(q)
-    wsbuf = api.alloc_workspace(B, H, N, d, w.mode, dev)
+    wsbuf = (api.alloc_workspace_blocksmooth if q_blocks else api.alloc_workspace)(B, H, N, d, w.mode, dev)
     nbytes = wsbuf.numel()
     stream = torch.cuda.current_stream()
 
     def step(ev):
         ev[0].record(stream)
-        api.sage_quantize_qkv(q, k, v, dcode, B, H, N, d, w.smooth_q, w.mode, wsbuf, nbytes, stream)
+        if q_blocks:
+            api.sage_quantize_qkv_blocksmooth(q, k, v, dcode, B, H, N, d, w.mode, wsbuf, nbytes, stream)
+        else:
+            api.sage_quantize_qkv(q, k, v, dcode, B, H, N, d, w.smooth_q, w.mode, wsbuf, nbytes, stream)
         ev[1].record(stream)
-        api.sage_attn_quantized(wsbuf, nbytes, out, dcode, B, H, N, d, w.causal, w.smooth_q, w.mode, stream)
+        if q_blocks:
+            api.sage_attn_quantized_blocksmooth(wsbuf, nbytes, out, dcode, B, H, N, d, w.causal, w.mode, stream)
+        else:
+            api.sage_attn_quantized(wsbuf, nbytes, out, dcode, B, H, N, d, w.causal, w.smooth_q, w.mode, stream)
         ev[2].record(stream)
 
     evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
@@ -364,7 +371,7 @@ def accuracy_leg(w, t, rows_n=48):
             "sample": "slice (b0,h0), %d evenly spaced query rows" % len(rows)}
 
 
-def e2e_leg(w, t, dev, steps, ws):
+def e2e_leg(w, t, dev, steps, ws, q_blocks=False):
     """End to end through the C ABI with host buffers (pinned): every step's
     host->device copy of Q, K, V and device->host copy of O are inside the
     timed region.  Steps are pipelined the way a serving loop runs them:
@@ -396,8 +403,12 @@ def e2e_leg(w, t, dev, steps, ws):
             stream.wait_event(ev_in[i])
             if i >= 2:
                 stream.wait_event(ev_out[i - 2])  # this slot's output has been copied out
-            api.sage_attn_fwd(dins[sl][0], dins[sl][1], dins[sl][2], douts[sl], B, H, N, d, w.causal, w.mode,
-                              t["dcode"], w.smooth_q, wsbuf, nbytes, stream)
+            if q_blocks:
+                api.sage_attn_fwd_blocksmooth(dins[sl][0], dins[sl][1], dins[sl][2], douts[sl], B, H, N, d,
+                                              w.causal, w.mode, t["dcode"], wsbuf, nbytes, stream)
+            else:
+                api.sage_attn_fwd(dins[sl][0], dins[sl][1], dins[sl][2], douts[sl], B, H, N, d, w.causal, w.mode,
+                                  t["dcode"], w.smooth_q, wsbuf, nbytes, stream)
             ev_c[i].record(stream)
             s_out.wait_event(ev_c[i])
             with torch.cuda.stream(s_out):
@@ -456,6 +467,66 @@ def fused_leg(w, dev, steps, warmup):
     return res
 
 
+def q_blocks_leg(w, dev, steps, warmup):
+    """Q smoothed per slice (sage_quantize_qkv + sage_attn_quantized with
+    smooth_q) against Q smoothed per 128-row block (the sage_*_blocksmooth
+    calls) on the same inputs: quantization and attention timed apart, CUDA
+    events on the launch stream, the two paths alternating (three rounds,
+    medians).  The per-block quantization adds the block means and one bias
+    row per block: Npad^2 * d / 128 fp32 multiply-adds per slice."""
+    w = inputs.variant(w, smooth_q=True)
+    B, H, N, d = w.shape()
+    dcode = api.DTYPE_CODE[inputs.DTYPES[w.dtype]]
+    q, k, v = [t.to(dev) for t in inputs.generate(w, device="cuda")]
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    ws_s = api.alloc_workspace(B, H, N, d, w.mode, dev)
+    ws_b = api.alloc_workspace_blocksmooth(B, H, N, d, w.mode, dev)
+    paths = {
+        "per_slice": (lambda: api.sage_quantize_qkv(q, k, v, dcode, B, H, N, d, True, w.mode, ws_s, ws_s.numel(),
+                                                    stream),
+                      lambda: api.sage_attn_quantized(ws_s, ws_s.numel(), out, dcode, B, H, N, d, w.causal, True,
+                                                      w.mode, stream)),
+        "per_block": (lambda: api.sage_quantize_qkv_blocksmooth(q, k, v, dcode, B, H, N, d, w.mode, ws_b,
+                                                                ws_b.numel(), stream),
+                      lambda: api.sage_attn_quantized_blocksmooth(ws_b, ws_b.numel(), out, dcode, B, H, N, d,
+                                                                  w.causal, w.mode, stream)),
+    }
+    for fq, fa in paths.values():
+        for _ in range(warmup):
+            fq()
+            fa()
+    times = {name: ([], []) for name in paths}
+    for _ in range(3):
+        for name, (fq, fa) in paths.items():
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+            for e in evs:
+                e[0].record(stream)
+                fq()
+                e[1].record(stream)
+                fa()
+                e[2].record(stream)
+            torch.cuda.synchronize()
+            times[name][0].append(float(np.mean([a.elapsed_time(b) for a, b, _ in evs])))
+            times[name][1].append(float(np.mean([b.elapsed_time(c) for _, b, c in evs])))
+    api.sage_check(ws_s, ws_s.numel(), stream)
+    api.sage_check(ws_b, ws_b.numel(), stream)
+    res = {}
+    for name, (tq, ta) in times.items():
+        res[name + "_quant_ms"] = float(np.median(tq))
+        res[name + "_attn_ms"] = float(np.median(ta))
+    Np = (N + 127) // 128 * 128
+    fma = B * H * (Np // 128) * Np * d
+    extra = res["per_block_quant_ms"] - res["per_slice_quant_ms"]
+    res["bias_fma_per_step"] = fma
+    res["bias_fma_rate_lower_bound_tfma_s"] = fma / (extra * 1e-3) / 1e12 if extra > 0 else None
+    res["value_per_block"] = inputs.attention_ops(w) / ((res["per_block_quant_ms"] + res["per_block_attn_ms"]) *
+                                                        1e-3) / 1e12
+    res["rounds"] = "3 alternating rounds of %d steps each, medians; the rate bound charges the whole extra " \
+                    "quantization time to the bias rows" % steps
+    return res
+
+
 def per_config_leg(dev, steps, probe, hbm, skip):
     names = ["sweep_N%d_d%d_%s" % (n, d, c) for d in (128, 64) for c in ("full", "causal")
              for n in (1024, 2048, 4096, 8192, 16384, 32768)]
@@ -482,6 +553,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the per-config sweep, the tensor-core probe and the accuracy leg")
+    ap.add_argument("--q-blocks", action="store_true",
+                    help="smooth Q per 128-row block (sage_*_blocksmooth calls; implies smooth_q)")
     ap.add_argument("--N", type=int, default=0,
                     help="override the workload's sequence length (small cases for profiling; "
                          "the headline runs use the workload's own N)")
@@ -492,6 +565,8 @@ def main():
     w = workload(args.workload)
     if args.N > 0:
         w = inputs.variant(w, N=args.N)
+    if args.q_blocks:
+        w = inputs.variant(w, smooth_q=True)
     ws, rank, local = replicas.init("nccl") if args.impl == "ours" or int(
         os.environ.get("WORLD_SIZE", "1")) > 1 else (1, 0, 0)
 
@@ -507,14 +582,14 @@ def main():
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     peaks, peak_src = load_peaks()
     hbm = peaks["hbm_gbs"]
-    extras = ws == 1 and not args.no_extras
+    extras = ws == 1 and not args.no_extras and not args.q_blocks
 
     # every rank probes its own GPU (no collective), so the roofline fraction
     # has the same denominator at every N
     probe = probe_peaks(dev, sm_count) if not args.no_extras else None
 
     clocks = ClockSampler(local)
-    t = time_workload(w, dev, args.steps, args.warmup, seed_rank=rank, clocks=clocks, ws=ws)
+    t = time_workload(w, dev, args.steps, args.warmup, seed_rank=rank, clocks=clocks, ws=ws, q_blocks=args.q_blocks)
     ms = replicas.max_over_ranks(t["ms"], ws, "cuda")
     attn_avg = replicas.max_over_ranks(t["attn_ms"], ws, "cuda")
     quant_avg = replicas.max_over_ranks(t["quant_ms"], ws, "cuda")
@@ -541,13 +616,16 @@ def main():
                 "traffic": traffic, "traffic_unit": "bytes per launch", "attn_ms": attn_avg,
                 "algorithmic_ops_per_launch": inputs.executed_ops(w)}
     qb = quant_bytes(w)
-    quant_line = {"bound": "hbm", "kernel": "quant_pass_kernel (stats) + quant_fold_kernel + quant_pass_kernel (codes)",
+    qkern = "quant_pass_kernel (stats) + quant_fold_kernel + quant_pass_kernel (codes)"
+    if args.q_blocks:
+        qkern += " + quant_fold_qblock_kernel + qblock_bias_kernel (bias rows not counted in the bytes)"
+    quant_line = {"bound": "hbm", "kernel": qkern,
                   "ms": quant_avg, "algorithmic_bytes": qb, "achieved": qb / (quant_avg * 1e-3) / 1e9,
                   "peak": hbm, "unit": "GB/s", "frac": qb / (quant_avg * 1e-3) / 1e9 / hbm,
                   "peak_source": "%s hbm_gbs" % peak_src}
 
     acc = accuracy_leg(w, t) if rank == 0 and extras else None
-    e2e = e2e_leg(w, t, dev, max(4, min(args.steps, 12)), ws)
+    e2e = e2e_leg(w, t, dev, max(4, min(args.steps, 12)), ws, q_blocks=args.q_blocks)
     clk = t["clocks"]
     del t
     torch.cuda.empty_cache()
@@ -559,18 +637,25 @@ def main():
         torch.cuda.empty_cache()
         fused["llm_prefill"] = fused_leg(workload("llm_prefill"), dev, 10, 3)
         torch.cuda.empty_cache()
+    q_blocks = None
+    if extras and w.mode != 2:
+        q_blocks = {}
+        for name in ("video_dit", "llm_prefill"):
+            q_blocks[name] = q_blocks_leg(workload(name), dev, 10, 3)
+            torch.cuda.empty_cache()
 
     line = {"metric": METRIC, "value": value,
             "unit": "TOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dtype_desc, "data": "synthetic",
-            "config": config_of(w, ws),
+            "config": config_of(w, ws, args.q_blocks),
             "value_executed": inputs.executed_ops(w) * ws / (ms * 1e-3) / 1e12,
             "roofline": roofline,
             "quant_roofline": quant_line,
             "e2e": e2e,
             # per step: the stats, fold and codes quantization kernels and the attention kernel
-            "gpu_launches": 4 * args.steps,
+            # (Q smoothed per block: also the block-mean fold and the bias rows)
+            "gpu_launches": (6 if args.q_blocks else 4) * args.steps,
             "clocks": clk}
     if probe is not None:
         line["tensor_peaks"] = probe
@@ -581,6 +666,9 @@ def main():
     if fused is not None:
         # Q quantized inside the attention kernel (sage_attn_fwd_fused), whole step
         line["fused_q"] = fused
+    if q_blocks is not None:
+        # Q smoothed per slice vs per 128-row block (sage_*_blocksmooth)
+        line["q_blocks"] = q_blocks
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle as orc
         orc.build()

@@ -226,6 +226,39 @@ SAGE_API sage_status sage_attn_fwd_gqa(const void* q, const void* k, const void*
                                        int Nq, int Nk, int d, int causal, int mode, int dtype, int smooth_q, void* ws,
                                        size_t ws_bytes, sage_stream_t stream);
 
+/* Q smoothed per block of 128 query rows instead of per slice.  The
+ * SageAttention2 abstract smooths Q by subtracting its channel mean but fixes
+ * no granularity for that mean; these calls take one mean per 128-row block
+ * (the attention's query tile), which follows Q where its offset drifts
+ * along the sequence.  Per slice and block b (rows 128b .. min(N, 128b+128)):
+ *   mean_b[c] = (sum over the block's 64-row chunks, in order, of the
+ *               sequential fp32 sum of the chunk) / (valid rows of the block);
+ *   the block's Q codes and 32-row granule scales as in sage_quantize_qkv,
+ *   after subtracting mean_b;
+ *   bias_b[j] = fma chain over c, in order, of mean_b[c] * (k - k_mean)[j, c]
+ *   for every key j < N (0 for padded keys); query row i adds the row of its
+ *   own block, bias_{i/128}.
+ * K, V and everything else as in sage_quantize_qkv / sage_attn_quantized with
+ * smooth_q = 1.  INT8/FP8 modes only (SAGE_MODE_NVFP4 returns
+ * SAGE_ERR_UNSUPPORTED).  Workspace layout (sage_workspace_layout_blocksmooth):
+ * the per-head layout with q_mean f32 [BH, Npad/128, d] and q_bias f32
+ * [BH, Npad/128, Npad].  The bias takes 4 * Npad^2 / 128 bytes per slice (32
+ * MiB at N = 32768) and Npad^2 * d / 128 fp32 multiply-adds on the CUDA
+ * cores (1/256 of the attention's tensor-core operations, run at a small
+ * fraction of their rate): on a B200 a quantize + attention step takes 7-9 %
+ * longer than with per-slice smoothing (B1 H12 N32760 d128 and B1 H32 N8192
+ * d128 causal).  Other arguments,
+ * alignment and error behaviour as for the per-head calls. */
+SAGE_API sage_status sage_workspace_layout_blocksmooth(int B, int H, int N, int d, int mode, sage_ws_layout* out);
+SAGE_API sage_status sage_quantize_qkv_blocksmooth(const void* q, const void* k, const void* v, int dtype, int B,
+                                                   int H, int N, int d, int mode, void* ws, size_t ws_bytes,
+                                                   sage_stream_t stream);
+SAGE_API sage_status sage_attn_quantized_blocksmooth(const void* ws, size_t ws_bytes, void* out, int dtype, int B,
+                                                     int H, int N, int d, int causal, int mode, sage_stream_t stream);
+SAGE_API sage_status sage_attn_fwd_blocksmooth(const void* q, const void* k, const void* v, void* out, int B, int H,
+                                               int N, int d, int causal, int mode, int dtype, void* ws,
+                                               size_t ws_bytes, sage_stream_t stream);
+
 /* Parity helper: the INT32 tile S = Q^ K^T of query tile `q_tile` and key tile
  * `k_tile` (128 x 128) of slice `bh`, computed by the same tensor-core path as
  * the attention kernel (kind::i8 MMA, accumulator in TMEM).  out: device

@@ -22,7 +22,9 @@ DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1}
 EXPORTED = ("sage_workspace_layout", "sage_workspace_size", "sage_quantize_qkv", "sage_quantize_qkv_static",
             "sage_attn_quantized",
             "sage_attn_fwd", "sage_attn_fwd_fused", "sage_attn_fwd_ranges", "sage_workspace_layout_gqa", "sage_quantize_qkv_gqa",
-            "sage_attn_quantized_gqa", "sage_attn_fwd_gqa", "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_probe_mma_rate",
+            "sage_attn_quantized_gqa", "sage_attn_fwd_gqa", "sage_workspace_layout_blocksmooth",
+            "sage_quantize_qkv_blocksmooth", "sage_attn_quantized_blocksmooth", "sage_attn_fwd_blocksmooth",
+            "sage_debug_qk_s32", "sage_debug_fp4_s", "sage_debug_timeout_probe", "sage_probe_mma_rate",
             "sage_check", "sage_last_error")
 PROBE_I8, PROBE_F8_F32ACC, PROBE_F8_F16ACC, PROBE_BF16, PROBE_FP4 = range(5)
 
@@ -76,6 +78,14 @@ def lib() -> ctypes.CDLL:
         L.sage_attn_quantized_gqa.restype = i
         L.sage_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.sage_attn_fwd_gqa.restype = i
+        L.sage_workspace_layout_blocksmooth.argtypes = [i, i, i, i, i, ctypes.POINTER(WsLayout)]
+        L.sage_workspace_layout_blocksmooth.restype = i
+        L.sage_quantize_qkv_blocksmooth.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_quantize_qkv_blocksmooth.restype = i
+        L.sage_attn_quantized_blocksmooth.argtypes = [vp, sz, vp, i, i, i, i, i, i, i, vp]
+        L.sage_attn_quantized_blocksmooth.restype = i
+        L.sage_attn_fwd_blocksmooth.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+        L.sage_attn_fwd_blocksmooth.restype = i
         L.sage_debug_qk_s32.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
         L.sage_debug_qk_s32.restype = i
         L.sage_debug_fp4_s.argtypes = [vp, sz, i, i, i, i, i, i, i, vp, vp]
@@ -199,6 +209,58 @@ def ws_views_gqa(ws: torch.Tensor, B, Hq, Hkv, Nq, Nk, d, mode) -> dict:
         k_mean=view(L.k_mean, BHk * d * 4, torch.float32, (BHk, d)),
         q_mean=view(L.q_mean, BHq * d * 4, torch.float32, (BHq, d)),
         q_bias=view(L.q_bias, BHq * Npk * 4, torch.float32, (BHq, Npk)),
+    )
+
+
+def sage_workspace_layout_blocksmooth(B, H, N, d, mode) -> WsLayout:
+    out = WsLayout()
+    _raise(lib().sage_workspace_layout_blocksmooth(B, H, N, d, mode, ctypes.byref(out)))
+    return out
+
+
+def sage_quantize_qkv_blocksmooth(q, k, v, dtype, B, H, N, d, mode, ws, ws_bytes, stream=None):
+    _raise(lib().sage_quantize_qkv_blocksmooth(_ptr(q), _ptr(k), _ptr(v), dtype, B, H, N, d, mode, _ptr(ws), ws_bytes,
+                                               _stream(stream)))
+
+
+def sage_attn_quantized_blocksmooth(ws, ws_bytes, out, dtype, B, H, N, d, causal, mode, stream=None):
+    _raise(lib().sage_attn_quantized_blocksmooth(_ptr(ws), ws_bytes, _ptr(out), dtype, B, H, N, d, int(causal), mode,
+                                                 _stream(stream)))
+
+
+def sage_attn_fwd_blocksmooth(q, k, v, out, B, H, N, d, causal, mode, dtype, ws, ws_bytes, stream=None):
+    _raise(lib().sage_attn_fwd_blocksmooth(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, int(causal), mode, dtype,
+                                           _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def alloc_workspace_blocksmooth(B, H, N, d, mode, device="cuda") -> torch.Tensor:
+    """Device workspace for the per-block Q smoothing calls (1024-byte aligned)."""
+    n = sage_workspace_layout_blocksmooth(B, H, N, d, mode).total
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 1024
+    return raw[off:off + n]
+
+
+def ws_views_blocksmooth(ws: torch.Tensor, B, H, N, d, mode) -> dict:
+    """Typed views of a per-block Q smoothing workspace: the per-head buffers
+    with q_mean [BH, Npad/128, d] and q_bias [BH, Npad/128, Npad]."""
+    L = sage_workspace_layout_blocksmooth(B, H, N, d, mode)
+    BH, Np = B * H, (N + 127) // 128 * 128
+    nb = Np // 128
+
+    def view(off, nbytes, dtype, shape):
+        return ws[off:off + nbytes].view(dtype).view(*shape)
+
+    return dict(
+        q_codes=view(L.q_codes, BH * Np * d, torch.int8, (BH, Np, d)),
+        k_codes=view(L.k_codes, BH * Np * d, torch.int8, (BH, Np, d)),
+        vt_codes=view(L.vt_codes, BH * d * Np, torch.uint8, (BH, d, Np)),
+        q_scale=view(L.q_scale, BH * (Np // 32) * 4, torch.float32, (BH, Np // 32)),
+        k_scale=view(L.k_scale, BH * (Np // 64) * 4, torch.float32, (BH, Np // 64)),
+        v_scale=view(L.v_scale, BH * d * 4, torch.float32, (BH, d)),
+        k_mean=view(L.k_mean, BH * d * 4, torch.float32, (BH, d)),
+        q_mean=view(L.q_mean, BH * nb * d * 4, torch.float32, (BH, nb, d)),
+        q_bias=view(L.q_bias, BH * nb * Np * 4, torch.float32, (BH, nb, Np)),
     )
 
 

@@ -52,11 +52,15 @@ sage_status check_shape_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int m
   return SAGE_OK;
 }
 
-sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode);
+// q_blocks: Q smoothed per 128-row block (per-head shapes): q_mean and q_bias
+// hold one row per block instead of one per slice.
+sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode, bool q_blocks = false);
 
-sage_ws_layout layout_of(int B, int H, int N, int d, int mode) { return layout_of_gqa(B, H, H, N, N, d, mode); }
+sage_ws_layout layout_of(int B, int H, int N, int d, int mode, bool q_blocks = false) {
+  return layout_of_gqa(B, H, H, N, N, d, mode, q_blocks);
+}
 
-sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode) {
+sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mode, bool q_blocks) {
   sage_ws_layout L;
   memset(&L, 0, sizeof(L));
   const bool split = Hq != Hkv || Nq != Nk;
@@ -87,8 +91,9 @@ sage_ws_layout layout_of_gqa(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
     L.global_scale = take(0);
   }
   L.k_mean = take(BHk * d * sizeof(float));
-  L.q_mean = take(BH * d * sizeof(float));
-  L.q_bias = take(BH * Npk * sizeof(float));
+  const size_t qrows = q_blocks ? Np / 128 : 1;  // mean and bias rows per slice
+  L.q_mean = take(BH * qrows * d * sizeof(float));
+  L.q_bias = take(BH * qrows * Npk * sizeof(float));
   // statistics partials and V multipliers of the quantize pass
   L.scratch = take((split ? sage::quant_scratch_floats_split((int)BH, (int)Np, (int)BHk, (int)Npk, d)
                           : sage::quant_scratch_floats((int)BH, (int)Np, d, mode)) *
@@ -216,10 +221,11 @@ static float default_vr(int mode) { return mode == SAGE_MODE_INT8_FP8_F16ACC ? 4
 static float default_pr(int mode) { return mode == SAGE_MODE_INT8_FP8_F16ACC ? 224.0f : 448.0f; }
 
 static sage_status quantize(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
-                            int smooth_q, int mode, float Vr, void* ws, size_t ws_bytes, sage_stream_t stream);
+                            int smooth_q, int mode, float Vr, void* ws, size_t ws_bytes, sage_stream_t stream,
+                            bool q_blocks = false);
 static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
                                   int causal, int smooth_q, int mode, float Pr, sage_stream_t stream,
-                                  bool after_quantize);
+                                  bool after_quantize, bool q_blocks = false);
 
 sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
                               int smooth_q, int mode, void* ws, size_t ws_bytes, sage_stream_t stream) {
@@ -227,16 +233,18 @@ sage_status sage_quantize_qkv(const void* q, const void* k, const void* v, int d
 }
 
 static sage_status quantize(const void* q, const void* k, const void* v, int dtype, int B, int H, int N, int d,
-                            int smooth_q, int mode, float Vr, void* ws, size_t ws_bytes, sage_stream_t stream) {
+                            int smooth_q, int mode, float Vr, void* ws, size_t ws_bytes, sage_stream_t stream,
+                            bool q_blocks) {
   sage_status st = check_shape(B, H, N, d, mode);
   if (st != SAGE_OK) return st;
   if (!q || !k || !v) return set_err(SAGE_ERR_INVALID_ARG, "null input pointer%s");
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
   if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v)) % 16)
     return set_err(SAGE_ERR_INVALID_ARG, "inputs must be 16-byte aligned%s");
-  const sage_ws_layout L = layout_of(B, H, N, d, mode);
+  const sage_ws_layout L = layout_of(B, H, N, d, mode, q_blocks);
   if ((st = check_ws(ws, ws_bytes, L.total)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, 0};
+  pb.q_blocks = q_blocks ? 1 : 0;
   if ((st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
   return cuda_status(sage::launch_quant_int8_fp8(q, k, v, pb, Vr, resolve(ws, L), (cudaStream_t)stream),
@@ -279,7 +287,7 @@ sage_status sage_quantize_qkv_static(const void* q, const void* k, const void* v
 // word is already clear; called on its own it clears it first.
 static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N, int d,
                                   int causal, int smooth_q, int mode, float Pr, sage_stream_t stream,
-                                  bool after_quantize) {
+                                  bool after_quantize, bool q_blocks) {
   sage_status st = check_shape(B, H, N, d, mode);
   if (st != SAGE_OK) return st;
   if (!out) return set_err(SAGE_ERR_INVALID_ARG, "null output pointer%s");
@@ -287,9 +295,10 @@ static sage_status attn_quantized(const void* ws, size_t ws_bytes, void* out, in
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return set_err(SAGE_ERR_INVALID_ARG, "dtype must be 0 (f16) or 1 (bf16)%s");
   if (mode == SAGE_MODE_NVFP4 && d != 128)
     return set_err(SAGE_ERR_UNSUPPORTED, "the NVFP4 attention kernel needs d = 128%s");
-  const sage_ws_layout L = layout_of(B, H, N, d, mode);
+  const sage_ws_layout L = layout_of(B, H, N, d, mode, q_blocks);
   if ((st = check_ws(ws, ws_bytes, L.scratch)) != SAGE_OK) return st;
   sage::Problem pb{B * H, N, (N + 127) / 128 * 128, d, dtype, smooth_q ? 1 : 0, mode, causal ? 1 : 0};
+  pb.q_blocks = q_blocks ? 1 : 0;
   if (!after_quantize &&
       (st = cuda_status(cudaMemsetAsync((char*)ws + L.error, 0, sizeof(int), (cudaStream_t)stream), "clear")) != SAGE_OK)
     return st;
@@ -434,6 +443,46 @@ sage_status sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void*
   st = sage_quantize_qkv_gqa(q, k, v, dtype, B, Hq, Hkv, Nq, Nk, d, smooth_q, mode, ws, ws_bytes, stream);
   if (st != SAGE_OK) return st;
   return attn_quantized_gqa(ws, ws_bytes, out, dtype, B, Hq, Hkv, Nq, Nk, d, causal, smooth_q, mode, stream, true);
+}
+
+// Q smoothed per 128-row block: the per-head entry points with smooth_q set
+// and one Q mean and one bias row per block.
+static sage_status check_blocksmooth(int B, int H, int N, int d, int mode) {
+  sage_status st = check_shape(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (mode == SAGE_MODE_NVFP4)
+    return set_err(SAGE_ERR_UNSUPPORTED, "per-block Q smoothing covers the INT8/FP8 modes%s");
+  return SAGE_OK;
+}
+
+sage_status sage_workspace_layout_blocksmooth(int B, int H, int N, int d, int mode, sage_ws_layout* out) {
+  sage_status st = check_blocksmooth(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  if (!out) return set_err(SAGE_ERR_INVALID_ARG, "layout pointer is null%s");
+  *out = layout_of(B, H, N, d, mode, true);
+  return SAGE_OK;
+}
+
+sage_status sage_quantize_qkv_blocksmooth(const void* q, const void* k, const void* v, int dtype, int B, int H, int N,
+                                          int d, int mode, void* ws, size_t ws_bytes, sage_stream_t stream) {
+  sage_status st = check_blocksmooth(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  return quantize(q, k, v, dtype, B, H, N, d, 1, mode, default_vr(mode), ws, ws_bytes, stream, true);
+}
+
+sage_status sage_attn_quantized_blocksmooth(const void* ws, size_t ws_bytes, void* out, int dtype, int B, int H, int N,
+                                            int d, int causal, int mode, sage_stream_t stream) {
+  sage_status st = check_blocksmooth(B, H, N, d, mode);
+  if (st != SAGE_OK) return st;
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, 1, mode, default_pr(mode), stream, false, true);
+}
+
+sage_status sage_attn_fwd_blocksmooth(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                                      int d, int causal, int mode, int dtype, void* ws, size_t ws_bytes,
+                                      sage_stream_t stream) {
+  sage_status st = sage_quantize_qkv_blocksmooth(q, k, v, dtype, B, H, N, d, mode, ws, ws_bytes, stream);
+  if (st != SAGE_OK) return st;
+  return attn_quantized(ws, ws_bytes, out, dtype, B, H, N, d, causal, 1, mode, default_pr(mode), stream, true, true);
 }
 
 sage_status sage_debug_qk_s32(const void* ws, size_t ws_bytes, int B, int H, int N, int d, int bh, int q_tile,

@@ -125,10 +125,14 @@ SAGE_DEV int kv_slice(const AttnArgs& a, int bh) {
 
 }  // namespace
 
-template <int D, typename OutT, bool HAS_BIAS, bool F16ACC, bool FUSED_Q>
+// BIAS: 0 none; 1 one bias row per slice ([BH][Npad_k]); 2 one row per
+// 128-row query tile ([BH][Npad/128][Npad_k], Q smoothed per block).
+template <int D, typename OutT, int BIAS, bool F16ACC, bool FUSED_Q>
 __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  static_assert(BIAS >= 0 && BIAS <= 2 && !(BIAS == 2 && FUSED_Q), "per-tile bias rows: two-step path only");
+  constexpr bool HAS_BIAS = BIAS != 0, kTileBias = BIAS == 2;
   using R = Roles<F16ACC>;
   constexpr int kNQ = R::kNQ;
   constexpr int kSoftmaxWarps = R::kSoftmaxWarps, kProducerWarp = R::kProducerWarp, kMmaWarp = R::kMmaWarp;
@@ -429,7 +433,9 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       const uint32_t t_h = tmem + lane_off + kColH;
       uint8_t* prow0 = smem + L::off_p + 2 * q * L::kP + r * 128;  // buffer 0; buffer 1 is kP further
       const float* ksc = a.k_scale + (size_t)kv_slice(a, bh) * (a.Npad_k / 64);
-      const float* bvec = HAS_BIAS ? a.bias + (size_t)bh * a.Npad_k + h * 64 : nullptr;
+      const float* bvec = !HAS_BIAS ? nullptr
+                          : a.bias + (kTileBias ? ((size_t)bh * (a.Npad / 128) + qt) * a.Npad_k : (size_t)bh * a.Npad_k) +
+                                h * 64;
       // m: running row max of the logits (log2 units); l: this half's running
       // sum of p' = p * Pr.
       float m = -INFINITY, l = 0.f;
@@ -459,9 +465,19 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       };
       // K scales of both 64-key granules of the tile, loaded one tile ahead
       float2 ks_next = *reinterpret_cast<const float2*>(ksc);
+      // A bias row of its own per query tile (Q smoothed per block) is read
+      // by this CTA alone, from DRAM: its lines (two per key half and tile)
+      // are prefetched into L2 two tiles ahead.  A row shared by the slice
+      // stays in L2 without it.
+      constexpr bool bias_prefetch = kTileBias;
+      if (bias_prefetch) {
+        prefetch_l2(bvec + 32 * (lane & 1));
+        if (nt[q] > 1) prefetch_l2(bvec + 128 + 32 * (lane & 1));
+      }
       for (int j = 0; ok && j < nt[q]; ++j) {
         const float2 ks = ks_next;
         if (j + 1 < nt[q]) ks_next = *reinterpret_cast<const float2*>(ksc + 2 * (j + 1));
+        if (bias_prefetch && j + 2 < nt[q]) prefetch_l2(bvec + (j + 2) * 128 + 32 * (lane & 1));
         const int kbase = j * 128 + h * 64;
         // visible keys of this row among the half's 64 form the prefix c < lim
         int lim = 64;
@@ -772,10 +788,10 @@ static bool make_pair_maps(const WsPtrs& w, const Problem& pb, CUtensorMap* mk, 
   return make_tmap_u8_nd(mk, w.k_codes, 5, kd, ks, kb, (int)D) && make_tmap_u8_nd(mv, w.vt_codes, 4, vd, vs, vb, 128);
 }
 
-template <int D, typename OutT, bool HAS_BIAS, bool F16ACC, bool FUSED_Q>
+template <int D, typename OutT, int BIAS, bool F16ACC, bool FUSED_Q>
 static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                             int BH, cudaStream_t s) {
-  auto kern = attn_i8f8_kernel<D, OutT, HAS_BIAS, F16ACC, FUSED_Q>;
+  auto kern = attn_i8f8_kernel<D, OutT, BIAS, F16ACC, FUSED_Q>;
   using L = Smem<D, Roles<F16ACC>::kNQ>;
   // set on every launch: the attribute is per device, and a cached flag would
   // be shared by host threads and devices
@@ -824,13 +840,17 @@ static cudaError_t launch_attn(const WsPtrs& w, const void* q_raw, void* out, co
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)pb.d));
   a.log2Pr = (float)log2((double)Pr);
   const bool bias = a.bias != nullptr;
+  if (pb.q_blocks && (fused || !bias)) return cudaErrorInvalidValue;
 #define SAGE_RUN(DD, TT, BB, FF, QQ) run_attn<DD, TT, BB, FF, QQ>(mq, mk, mv, a, pb.BH, s)
 #define SAGE_RUN_Q(DD, TT, BB, FF) (fused ? SAGE_RUN(DD, TT, BB, FF, true) : SAGE_RUN(DD, TT, BB, FF, false))
 #define SAGE_RUN_F(DD, TT, BB) (f16 ? SAGE_RUN_Q(DD, TT, BB, true) : SAGE_RUN_Q(DD, TT, BB, false))
-#define SAGE_RUN_B(DD, TT) (bias ? SAGE_RUN_F(DD, TT, true) : SAGE_RUN_F(DD, TT, false))
+  // per-tile bias rows: the two-step path only (the fused Q prologue subtracts one mean per slice)
+#define SAGE_RUN_T(DD, TT) (f16 ? SAGE_RUN(DD, TT, 2, true, false) : SAGE_RUN(DD, TT, 2, false, false))
+#define SAGE_RUN_B(DD, TT) (!bias ? SAGE_RUN_F(DD, TT, 0) : pb.q_blocks ? SAGE_RUN_T(DD, TT) : SAGE_RUN_F(DD, TT, 1))
   if (pb.d == 128) return pb.dtype == 0 ? SAGE_RUN_B(128, __half) : SAGE_RUN_B(128, __nv_bfloat16);
   return pb.dtype == 0 ? SAGE_RUN_B(64, __half) : SAGE_RUN_B(64, __nv_bfloat16);
 #undef SAGE_RUN_B
+#undef SAGE_RUN_T
 #undef SAGE_RUN_F
 #undef SAGE_RUN_Q
 #undef SAGE_RUN

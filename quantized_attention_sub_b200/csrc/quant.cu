@@ -90,6 +90,9 @@ struct QuantArgs {
   // key/value slice, reading their means from q_mean_g.
   int roles, G;
   const float* q_mean_g;
+  // Q smoothed per 128-row block: the codes pass reads block blk / 2's mean
+  // from q_mean [BH][Npad/128][d] and writes no bias (qblock_bias_kernel does)
+  int q_blocks;
 };
 constexpr int kRolesQ = 1, kRolesKV = 2;
 
@@ -282,7 +285,10 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
         // the slice's means and V multipliers (written by the fold kernel)
         float* sl = reinterpret_cast<float*>(sm + L::kTiles) + b * (3 * D);
         if (do_kv || FP4) bulk_load(sl, a.k_mean + (size_t)bh * D, D * 4, &full[b]);
-        if (a.smooth_q && (do_q || FP4)) bulk_load(sl + D, a.q_mean + (size_t)bh * D, D * 4, &full[b]);
+        if (a.smooth_q && (do_q || FP4)) {
+          const size_t mrow = a.q_blocks ? (size_t)bh * (a.Npad / 128) + (blk >> 1) : (size_t)bh;
+          bulk_load(sl + D, a.q_mean + mrow * D, D * 4, &full[b]);
+        }
         if (FP4)
           bulk_load(sl + 2 * D, a.gscale + (size_t)bh * 4, 16, &full[b]);
         else if (do_kv)
@@ -666,7 +672,8 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
             }
           }
         }
-        if (a.smooth_q && do_kv && tid < kTok && do_q) {
+        const bool pass_bias = a.smooth_q && !a.q_blocks && do_kv && tid < kTok;
+        if (pass_bias && do_q) {
           // Q-smoothing bias of token t0 + tid: fma chain over channels of
           // mean_q[c] * k~[c] in channel order (k~ recomputed from the tile)
           const int row = tid;
@@ -687,7 +694,7 @@ __global__ void __launch_bounds__(kThreadsQ, 2) quant_pass_kernel(const __grid_c
             }
           }
           a.q_bias[(size_t)bh * a.Npad + t0 + row] = acc;
-        } else if (a.smooth_q && do_kv && tid < kTok) {
+        } else if (pass_bias) {
           // K/V pass with its own query heads: the bias of each of the G query
           // heads of this key/value slice (query slice bh * G + g), the same
           // chain with that head's mean read from global memory
@@ -848,6 +855,133 @@ __global__ void __launch_bounds__(D) quant_fold_kernel(const QuantArgs a) {
   }
 }
 
+// Q smoothed per 128-row block: block b = blockIdx.x of slice bh =
+// blockIdx.y, thread c = channel.  Its mean is the per-slice mean's chain
+// applied to the block's valid rows: the sum of the Q-sum partials of its
+// chunks 2b and 2b + 1 (the second only if it holds valid rows), in order,
+// from 0, divided by the number of valid rows.
+template <int D>
+__global__ void __launch_bounds__(D) quant_fold_qblock_kernel(const QuantArgs a) {
+  const int b = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  const int nchunks = a.Npad / 64, nblk = a.Npad / 128;
+  // launched while the fold kernel may still run: the statistics pass it
+  // waited for wrote the partials
+  grid_dep_wait();
+  grid_dep_launch();
+  // plane 1 of the partials: Q sums [BH][Npad/64][D]
+  const float* p = a.part + ((size_t)a.BH * nchunks + (size_t)bh * nchunks + 2 * b) * D + c;
+  const int r0 = 128 * b, rows = min(128, a.N - r0);
+  float acc = __fadd_rn(0.f, p[0]);
+  if (r0 + 64 < a.N) acc = __fadd_rn(acc, p[D]);
+  a.q_mean[((size_t)bh * nblk + b) * D + c] = __fdiv_rn(acc, (float)rows);
+}
+
+// Per-block Q-smoothing bias: q_bias[bh][b][j] = the fma chain over channels
+// c, in order and from 0, of mean_b[c] * RN(k[j][c] - k_mean[c]) -- the
+// per-slice bias with block b's mean -- for keys j < N, and 0 for the
+// padding.  A CTA computes 64 blocks x 128 keys of one slice (grid: key
+// tiles, block groups, slices) from shared-memory fp32 copies of k~ for its
+// keys and of the blocks' means, each row padded by 4 floats so that the
+// 16-byte loads of 8 consecutive lanes fall in distinct bank groups.  Warp w
+// owns blocks 8w .. 8w+7 of the group, lane l the keys l + 32 q, q < 4.
+constexpr int kBiasKeys = 128, kBiasBlocks = 64, kBiasThreads = 256;
+
+template <int D>
+constexpr size_t bias_smem_bytes() {
+  return (size_t)(kBiasKeys + kBiasBlocks) * (D + 4) * sizeof(float);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kBiasThreads, 2) qblock_bias_kernel(const T* __restrict__ k, const QuantArgs a) {
+  constexpr int RS = D + 4;  // floats per shared row
+  extern __shared__ __align__(16) float bsm[];
+  float* const kt = bsm;                     // [kBiasKeys][RS]
+  float* const mb = bsm + kBiasKeys * RS;    // [kBiasBlocks][RS]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j0 = blockIdx.x * kBiasKeys, b0 = blockIdx.y * kBiasBlocks, bh = blockIdx.z;
+  const int nblk = a.Npad / 128;
+  // the K means and block means come from the kernels before this one
+  grid_dep_wait();
+  grid_dep_launch();
+  {
+    // k~ of the CTA's keys and the group's block means (0 past the last
+    // block).  Every global load is issued before the first is used: each
+    // thread holds KIT 16-byte pieces of K (8 channels, always channels c0 ..
+    // c0 + 7) and MIT float4 of the means.
+    constexpr int PPR = D / 8, QPR = D / 4;
+    constexpr int KIT = kBiasKeys * PPR / kBiasThreads, MIT = kBiasBlocks * QPR / kBiasThreads;
+    static_assert(kBiasThreads % PPR == 0 && kBiasThreads % QPR == 0, "fixed column per thread");
+    const int c0 = 8 * (tid % PPR), r0 = tid / PPR;
+    const float* km = a.k_mean + (size_t)bh * D + c0;
+    const float4 km0 = __ldg(reinterpret_cast<const float4*>(km)), km1 = __ldg(reinterpret_cast<const float4*>(km + 4));
+    uint4 kraw[KIT];
+#pragma unroll
+    for (int it = 0; it < KIT; ++it) {
+      const int j = j0 + r0 + it * (kBiasThreads / PPR);
+      kraw[it] = j < a.N ? __ldg(reinterpret_cast<const uint4*>(k + ((size_t)bh * a.N + j) * D + c0))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const int mc0 = 4 * (tid % QPR), mr0 = tid / QPR;
+    float4 mraw[MIT];
+#pragma unroll
+    for (int it = 0; it < MIT; ++it) {
+      const int b = b0 + mr0 + it * (kBiasThreads / QPR);
+      mraw[it] = b < nblk ? __ldg(reinterpret_cast<const float4*>(a.q_mean + ((size_t)bh * nblk + b) * D + mc0))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float kmv[8] = {km0.x, km0.y, km0.z, km0.w, km1.x, km1.y, km1.z, km1.w};
+#pragma unroll
+    for (int it = 0; it < KIT; ++it) {
+      const int r = r0 + it * (kBiasThreads / PPR);
+      float x[8];
+      const uint32_t w4[4] = {kraw[it].x, kraw[it].y, kraw[it].z, kraw[it].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) unpack2<T>(w4[e], x[2 * e], x[2 * e + 1]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = j0 + r < a.N ? __fsub_rn(x[e], kmv[e]) : 0.f;
+      *reinterpret_cast<float4*>(kt + r * RS + c0) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(kt + r * RS + c0 + 4) = make_float4(x[4], x[5], x[6], x[7]);
+    }
+#pragma unroll
+    for (int it = 0; it < MIT; ++it)
+      *reinterpret_cast<float4*>(mb + (mr0 + it * (kBiasThreads / QPR)) * RS + mc0) = mraw[it];
+  }
+  __syncthreads();
+  const int bw = b0 + 8 * warp;  // this warp's first block
+  if (bw >= nblk) return;
+  float acc[8][4];
+#pragma unroll
+  for (int m = 0; m < 8; ++m)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
+#pragma unroll 2
+  for (int c0 = 0; c0 < D; c0 += 4) {
+    float4 kv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) kv[q] = *reinterpret_cast<const float4*>(kt + (lane + 32 * q) * RS + c0);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const float4 mv = *reinterpret_cast<const float4*>(mb + (8 * warp + m) * RS + c0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float t = acc[m][q];
+        t = __fmaf_rn(mv.x, kv[q].x, t);
+        t = __fmaf_rn(mv.y, kv[q].y, t);
+        t = __fmaf_rn(mv.z, kv[q].z, t);
+        t = __fmaf_rn(mv.w, kv[q].w, t);
+        acc[m][q] = t;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    if (bw + m >= nblk) break;
+    float* o = a.q_bias + ((size_t)bh * nblk + bw + m) * a.Npad + j0 + lane;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o[32 * q] = j0 + lane + 32 * q < a.N ? acc[m][q] : 0.f;
+  }
+}
+
 // NVFP4.  Per slice and tensor (blockIdx.y: 0 K, 1 V, 2 Q): the means (K;
 // Q with smooth_q) and the global scale g = A / (6 * 448), A = the slice's
 // max |x~| over valid tokens.  RN(x - mean) is monotone in x, so per channel
@@ -970,6 +1104,7 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
   a.roles = kRolesQ | kRolesKV;
   a.G = 1;
   a.q_mean_g = w.q_mean;
+  a.q_blocks = pb.q_blocks;
 
   // 16-bit [BH][N][D] inputs seen as bytes: rows of 2D bytes, boxes of
   // 128 bytes x 64 tokens (rows past N read as zero)
@@ -1001,10 +1136,24 @@ cudaError_t quant_run(const void* q, const void* k, const void* v, const Problem
   if (FP4)
     e = launch_kernel(quant_fold_fp4_kernel<D>, dim3(pb.BH, 3), dim3(D), 0, s, true, a);
   else
-    e = launch_kernel(quant_fold_kernel<D>, dim3(pb.BH, pb.smooth_q ? 3 : 2), dim3(D), 0, s, true, a);
+    e = launch_kernel(quant_fold_kernel<D>, dim3(pb.BH, pb.smooth_q && !pb.q_blocks ? 3 : 2), dim3(D), 0, s, true, a);
   if (e != cudaSuccess) return e;
-  return launch_kernel(quant_pass_kernel<T, D, kCodesPass, FP4>, dim3(g1), dim3(kThreadsQ), smem, s, true, tq, tk,
-                       tv, a);
+  const int nblk = pb.Npad / 128;
+  if (!FP4 && pb.q_blocks) {
+    // Q means per 128-row block (the fold above did K and V only)
+    e = launch_kernel(quant_fold_qblock_kernel<D>, dim3(nblk, pb.BH), dim3(D), 0, s, true, a);
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_kernel(quant_pass_kernel<T, D, kCodesPass, FP4>, dim3(g1), dim3(kThreadsQ), smem, s, true, tq, tk, tv,
+                    a);
+  if (e != cudaSuccess || FP4 || !pb.q_blocks) return e;
+  // the bias rows of the blocks (after the codes pass, which rereads the
+  // inputs the statistics pass left in L2)
+  const size_t bsmem = bias_smem_bytes<D>();
+  e = cudaFuncSetAttribute(qblock_bias_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(qblock_bias_kernel<T, D>, dim3(pb.Npad / kBiasKeys, (nblk + kBiasBlocks - 1) / kBiasBlocks, pb.BH),
+                       dim3(kBiasThreads), bsmem, s, true, static_cast<const T*>(k), a);
 }
 
 // Grouped key/value heads and / or separate query and key lengths (INT8/FP8
@@ -1040,6 +1189,7 @@ cudaError_t quant_run_split(const void* q, const void* k, const void* v, const P
   a.Vr = Vr;
   a.G = pb.G;
   a.q_mean_g = w.q_mean;
+  a.q_blocks = 0;
   QuantArgs aq = a, akv = a;
   aq.roles = kRolesQ;
   aq.BH = BHq;

@@ -31,6 +31,9 @@ struct WsPtrs {
 struct Problem {
   int BH, N, Npad, d, dtype, smooth_q, mode, causal;
   int Hq = 0, G = 1, Nk = 0, Npad_k = 0;
+  // Q smoothed per 128-row block (per-head shapes, INT8/FP8 modes): q_mean
+  // [BH][Npad/128][d] and q_bias [BH][Npad/128][Npad], one row per block
+  int q_blocks = 0;
   int nk() const { return Nk ? Nk : N; }
   int npk() const { return Npad_k ? Npad_k : Npad; }
   int bh_kv() const { return BH / G; }

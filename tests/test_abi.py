@@ -103,3 +103,24 @@ def test_gqa_causal_needs_nq_le_nk(lib):
     st = lib.sage_attn_fwd_gqa(vp(4096), vp(4096), vp(4096), vp(4096), 1, 4, 2, 300, 200, 64, 1, 0, 0, 0, vp(4096), ws,
                                vp(0))
     assert st == api.SAGE_ERR_UNSUPPORTED
+
+
+def test_blocksmooth_layout_holds_a_row_per_block(lib):
+    """The per-block Q smoothing layout is the per-head one with q_mean and
+    q_bias grown to one row per 128-row block; the NVFP4 mode is refused."""
+    for (B, H, N, d, mode) in [(1, 2, 300, 128, 0), (2, 3, 8300, 64, 1), (1, 1, 1, 64, 0)]:
+        a, b = api.sage_workspace_layout(B, H, N, d, mode), api.sage_workspace_layout_blocksmooth(B, H, N, d, mode)
+        Np = (N + 127) // 128 * 128
+        nb = Np // 128
+        for f in ("q_codes", "k_codes", "vt_codes", "q_scale", "k_scale", "v_scale", "k_mean", "q_mean"):
+            assert getattr(a, f) == getattr(b, f), f
+        assert b.q_bias - b.q_mean >= B * H * nb * d * 4
+        assert b.scratch - b.q_bias >= B * H * nb * Np * 4
+        offs = [getattr(b, f) for f, _ in api.WsLayout._fields_ if f != "total"]
+        assert all(o % 1024 == 0 for o in offs) and b.total > b.scratch
+    out = api.WsLayout()
+    assert lib.sage_workspace_layout_blocksmooth(1, 2, 300, 128, 2, ctypes.byref(out)) == api.SAGE_ERR_UNSUPPORTED
+    vp = ctypes.c_void_p
+    st = lib.sage_attn_fwd_blocksmooth(vp(4096), vp(4096), vp(4096), vp(4096), 1, 2, 300, 128, 0, 2, 0, vp(4096),
+                                       1 << 30, vp(0))
+    assert st == api.SAGE_ERR_UNSUPPORTED
