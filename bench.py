@@ -467,6 +467,74 @@ def fused_leg(w, dev, steps, warmup):
     return res
 
 
+def visible_pairs(Nq, Nk, causal):
+    """(query, key) pairs a slice computes: all Nq * Nk, or under the causal
+    mask aligned to the last key (query row i sees keys j <= i + Nk - Nq)
+    sum over i of min(Nk, i + Nk - Nq + 1)."""
+    if not causal:
+        return Nq * Nk
+    koff = Nk - Nq
+    # rows with i + koff + 1 < Nk see i + koff + 1 keys; the rest see Nk
+    full_from = max(0, Nk - koff - 1)
+    n_part = min(Nq, full_from)
+    part = n_part * (koff + 1) + n_part * (n_part - 1) // 2
+    return part + (Nq - n_part) * Nk
+
+
+GQA_CASES = (
+    # (name, base workload for the value law, B, Hq, Hkv, Nq, Nk, causal)
+    ("llm_prefill_gqa4", "llm_prefill", 1, 32, 8, 8192, 8192, True),
+    ("chunked_prefill_gqa4", "llm_prefill", 1, 32, 8, 2048, 32768, True),
+)
+
+
+def gqa_leg(dev, steps, warmup, probe):
+    """Grouped key/value heads and separate lengths (sage_*_gqa): quantization
+    and attention timed apart with CUDA events on the launch stream, inputs
+    drawn from the workload's value law (Q with Hq heads and Nq rows, K and V
+    with Hkv heads and Nk rows).  Operations count the visible pairs."""
+    res = {}
+    for name, base, B, Hq, Hkv, Nq, Nk, causal in GQA_CASES:
+        w0 = workload(base)
+        q = inputs.generate(inputs.variant(w0, B=B, H=Hq, N=Nq), device="cuda")[0].to(dev)
+        _, k, v = inputs.generate(inputs.variant(w0, B=B, H=Hkv, N=Nk, seed=w0.seed + 1), device="cuda")
+        k, v = k.to(dev), v.to(dev)
+        d = q.shape[-1]
+        dcode = api.DTYPE_CODE[q.dtype]
+        out = torch.empty_like(q)
+        wsbuf = api.alloc_workspace_gqa(B, Hq, Hkv, Nq, Nk, d, w0.mode, dev)
+        stream = torch.cuda.current_stream()
+        fq = lambda: api.sage_quantize_qkv_gqa(q, k, v, dcode, B, Hq, Hkv, Nq, Nk, d, False, w0.mode, wsbuf,
+                                               wsbuf.numel(), stream)
+        fa = lambda: api.sage_attn_quantized_gqa(wsbuf, wsbuf.numel(), out, dcode, B, Hq, Hkv, Nq, Nk, d, causal,
+                                                 False, w0.mode, stream)
+        for _ in range(warmup):
+            fq()
+            fa()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in evs:
+            e[0].record(stream)
+            fq()
+            e[1].record(stream)
+            fa()
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        api.sage_check(wsbuf, wsbuf.numel(), stream)
+        quant_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in evs]))
+        attn_ms = float(np.mean([b.elapsed_time(c) for _, b, c in evs]))
+        ops = 4.0 * B * Hq * visible_pairs(Nq, Nk, causal) * d
+        r = {"B": B, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "d": d, "dtype": w0.dtype, "causal": causal,
+             "mode": MODE_NAMES[w0.mode], "quant_ms": quant_ms, "attn_ms": attn_ms,
+             "attn_tops_executed": ops / (attn_ms * 1e-3) / 1e12,
+             "step_tops_executed": ops / ((quant_ms + attn_ms) * 1e-3) / 1e12}
+        if probe is not None:
+            r["attn_frac_of_probe_burst"] = r["attn_tops_executed"] / mode_peak(w0.mode, probe, "burst")
+        res[name] = r
+        del q, k, v, out, wsbuf
+        torch.cuda.empty_cache()
+    return res
+
+
 def q_blocks_leg(w, dev, steps, warmup):
     """Q smoothed per slice (sage_quantize_qkv + sage_attn_quantized with
     smooth_q) against Q smoothed per 128-row block (the sage_*_blocksmooth
@@ -637,6 +705,7 @@ def main():
         torch.cuda.empty_cache()
         fused["llm_prefill"] = fused_leg(workload("llm_prefill"), dev, 10, 3)
         torch.cuda.empty_cache()
+    gqa = gqa_leg(dev, 10, 3, probe) if extras else None
     q_blocks = None
     if extras and w.mode != 2:
         q_blocks = {}
@@ -669,6 +738,9 @@ def main():
     if q_blocks is not None:
         # Q smoothed per slice vs per 128-row block (sage_*_blocksmooth)
         line["q_blocks"] = q_blocks
+    if gqa is not None:
+        # grouped key/value heads and separate query / key lengths (sage_*_gqa)
+        line["gqa"] = gqa
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle as orc
         orc.build()

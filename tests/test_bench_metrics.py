@@ -41,3 +41,14 @@ def test_quantization_bytes(N, d, mode):
     reads = 3 * 2 * N * d * 2
     codes = 3 * 2 * Np * d * (0.5 + 1.0 / 16) if mode == 2 else 3 * 2 * Np * d
     assert b.quant_bytes(w) == reads + codes
+
+
+@pytest.mark.parametrize("Nq,Nk,causal", [(1, 1, True), (5, 5, True), (3, 10, True), (7, 130, True), (128, 128, False),
+                                           (2048, 4096, True), (10, 3, False)])
+def test_visible_pairs_match_brute_force(Nq, Nk, causal):
+    """Pairs the grouped-head leg counts: query row i sees keys j <= i + Nk - Nq
+    under the causal mask (aligned to the last key), every key otherwise."""
+    b = _bench()
+    i, j = np.meshgrid(np.arange(Nq), np.arange(Nk), indexing="ij")
+    brute = int(np.count_nonzero(j <= i + (Nk - Nq))) if causal else Nq * Nk
+    assert b.visible_pairs(Nq, Nk, causal) == brute
