@@ -157,3 +157,45 @@ def test_full_size_video_dit_blocksmooth_sampled():
         ref32, flip = orc.attention_int8_fp8(view, False, rows=rows, with_flip=True)
         got = out.float().cpu().reshape(B * H, N, d).numpy()[:, rows]
         compare_out(got, ref32, flip, "fp16", ("video_dit_blocksmooth", int(b)))
+
+
+def test_sweep_point_blocksmooth_sampled():
+    """The shape `bench.py --q-blocks` times (B4 H32 N8192 d128 fp16, FP32
+    accumulator, non-causal): on three of the 128 slices, K and V codes and
+    scales bit-exact; on sampled blocks of those slices the block means, Q
+    codes, scales and bias rows bit-exact (the oracle's per-block steps), and
+    the output on rows of those blocks."""
+    w = inputs.variant(inputs.sweep(8192, 128, False), smooth_q=True)
+    B, H, N, d = w.shape()
+    q, k, v = [t.cuda() for t in inputs.generate(w, device="cuda")]
+    ws = api.alloc_workspace_blocksmooth(B, H, N, d, 0)
+    out = torch.empty_like(q)
+    api.sage_attn_fwd_blocksmooth(q, k, v, out, B, H, N, d, False, 0, 0, ws, ws.numel())
+    api.sage_check(ws, ws.numel())
+    slices = np.array([0, 77, 127])
+    views = api.ws_views_blocksmooth(ws, B, H, N, d, 0)
+    g = {n: views[n][slices].cpu().numpy() for n in views}
+    f = lambda t: t.reshape(B * H, N, d)[slices].float().cpu().numpy()
+    qn, kn, vn = f(q), f(k), f(v)
+    oz = orc.quantize_int8_fp8(qn, kn, vn, smooth_q=False, mode=0)
+    for name in ("k_codes", "vt_codes"):
+        assert np.array_equal(g[name].view(np.uint8), oz[name].view(np.uint8)), name
+    for name in ("k_scale", "v_scale", "k_mean"):
+        assert np.array_equal(g[name].view(np.uint32), oz[name].view(np.uint32)), name
+    got_all = out.reshape(B * H, N, d)[slices].float().cpu().numpy()
+    qc, sq = np.zeros_like(oz["q_codes"]), np.zeros_like(oz["q_scale"])
+    for b in (0, 1, 31, 63):
+        r0 = 128 * b
+        mb = orc.channel_mean(np.ascontiguousarray(qn[:, r0:r0 + 128]))
+        assert np.array_equal(g["q_mean"][:, b].view(np.uint32), mb.view(np.uint32)), b
+        cb, sb = orc.quant_int8(np.ascontiguousarray(qn[:, r0:r0 + 128]), mb, orc.Q_GRANULE)
+        qc[:, r0:r0 + 128], sq[:, r0 // 32:r0 // 32 + 4] = cb, sb
+        assert np.array_equal(g["q_codes"][:, r0:r0 + 128], cb), b
+        assert np.array_equal(g["q_scale"][:, r0 // 32:r0 // 32 + 4].view(np.uint32), sb.view(np.uint32)), b
+        bias = orc.q_bias(kn, oz["k_mean"], mb)
+        assert np.array_equal(g["q_bias"][:, b].view(np.uint32), bias.view(np.uint32)), b
+        # rows of block b read only block b's Q codes and scales
+        view = dict(oz, q_codes=qc, q_scale=sq, q_bias=bias)
+        rows = np.array([r0, r0 + 63, r0 + 127], np.int32)
+        ref32, flip = orc.attention_int8_fp8(view, False, rows=rows, with_flip=True)
+        compare_out(got_all[:, rows], ref32, flip, "fp16", ("sweep_N8192_blocksmooth", b))
