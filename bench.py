@@ -693,7 +693,9 @@ def main():
                   "peak_source": "%s hbm_gbs" % peak_src}
 
     acc = accuracy_leg(w, t) if rank == 0 and extras else None
-    e2e = e2e_leg(w, t, dev, max(4, min(args.steps, 12)), ws, q_blocks=args.q_blocks)
+    # up to 20 pipelined steps: the first copy-in and the last compute and
+    # copy-out are not overlapped, a fixed cost that more steps amortize
+    e2e = e2e_leg(w, t, dev, max(4, min(args.steps, 20)), ws, q_blocks=args.q_blocks)
     clk = t["clocks"]
     del t
     torch.cuda.empty_cache()
