@@ -242,7 +242,9 @@ SAGE_API sage_status sage_attn_fwd_gqa(const void* q, const void* k, const void*
  * smooth_q = 1.  INT8/FP8 modes only (SAGE_MODE_NVFP4 returns
  * SAGE_ERR_UNSUPPORTED).  Workspace layout (sage_workspace_layout_blocksmooth):
  * the per-head layout with q_mean f32 [BH, Npad/128, d] and q_bias f32
- * [BH, Npad/128, Npad].  The bias takes 4 * Npad^2 / 128 bytes per slice (32
+ * stored key-tile-major, [BH, Npad/128 key tiles, Npad/128 blocks, 128]:
+ * block b's bias at key j is element ((bh * Npad/128 + j/128) * Npad/128 +
+ * b) * 128 + j % 128.  The bias takes 4 * Npad^2 / 128 bytes per slice (32
  * MiB at N = 32768) and Npad^2 * d / 128 fp32 multiply-adds on the CUDA
  * cores (1/256 of the attention's tensor-core operations, run at a small
  * fraction of their rate): on a B200 a quantize + attention step takes 7-9 %

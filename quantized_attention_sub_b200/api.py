@@ -243,7 +243,9 @@ def alloc_workspace_blocksmooth(B, H, N, d, mode, device="cuda") -> torch.Tensor
 
 def ws_views_blocksmooth(ws: torch.Tensor, B, H, N, d, mode) -> dict:
     """Typed views of a per-block Q smoothing workspace: the per-head buffers
-    with q_mean [BH, Npad/128, d] and q_bias [BH, Npad/128, Npad]."""
+    with q_mean [BH, Npad/128, d], and q_bias as [BH, Npad/128 blocks, Npad]
+    (a copy: the workspace stores the rows key-tile-major, [BH][key tile]
+    [block][128])."""
     L = sage_workspace_layout_blocksmooth(B, H, N, d, mode)
     BH, Np = B * H, (N + 127) // 128 * 128
     nb = Np // 128
@@ -260,7 +262,8 @@ def ws_views_blocksmooth(ws: torch.Tensor, B, H, N, d, mode) -> dict:
         v_scale=view(L.v_scale, BH * d * 4, torch.float32, (BH, d)),
         k_mean=view(L.k_mean, BH * d * 4, torch.float32, (BH, d)),
         q_mean=view(L.q_mean, BH * nb * d * 4, torch.float32, (BH, nb, d)),
-        q_bias=view(L.q_bias, BH * nb * Np * 4, torch.float32, (BH, nb, Np)),
+        q_bias=view(L.q_bias, BH * nb * Np * 4, torch.float32, (BH, nb, nb, 128)).permute(0, 2, 1, 3)
+        .reshape(BH, nb, Np),
     )
 
 

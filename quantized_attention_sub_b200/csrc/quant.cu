@@ -876,7 +876,8 @@ __global__ void __launch_bounds__(D) quant_fold_qblock_kernel(const QuantArgs a)
   a.q_mean[((size_t)bh * nblk + b) * D + c] = __fdiv_rn(acc, (float)rows);
 }
 
-// Per-block Q-smoothing bias: q_bias[bh][b][j] = the fma chain over channels
+// Per-block Q-smoothing bias: bias row b of slice bh at key j (stored at
+// q_bias[bh][j / 128][b][j % 128], key-tile-major) = the fma chain over channels
 // c, in order and from 0, of mean_b[c] * RN(k[j][c] - k_mean[c]) -- the
 // per-slice bias with block b's mean -- for keys j < N, and 0 for the
 // padding.  A CTA computes 64 blocks x 128 keys of one slice (grid: key
@@ -976,7 +977,8 @@ __global__ void __launch_bounds__(kBiasThreads, 2) qblock_bias_kernel(const T* _
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
     if (bw + m >= nblk) break;
-    float* o = a.q_bias + ((size_t)bh * nblk + bw + m) * a.Npad + j0 + lane;
+    // key-tile-major: [BH][key tile][block][128 keys]
+    float* o = a.q_bias + (((size_t)bh * nblk + blockIdx.x) * nblk + bw + m) * kBiasKeys + lane;
 #pragma unroll
     for (int q = 0; q < 4; ++q) o[32 * q] = j0 + lane + 32 * q < a.N ? acc[m][q] : 0.f;
   }

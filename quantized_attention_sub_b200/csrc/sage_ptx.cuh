@@ -93,6 +93,8 @@ SAGE_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents
 // ---------------------------------------------------------------- TMA
 // Bring the line holding global address `p` into L2 (no result, no wait).
 SAGE_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// The same into L1.
+SAGE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 SAGE_DEV void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
