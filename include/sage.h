@@ -247,9 +247,9 @@ SAGE_API sage_status sage_attn_fwd_gqa(const void* q, const void* k, const void*
  * b) * 128 + j % 128.  The bias takes 4 * Npad^2 / 128 bytes per slice (32
  * MiB at N = 32768) and Npad^2 * d / 128 fp32 multiply-adds on the CUDA
  * cores (1/256 of the attention's tensor-core operations, run at a small
- * fraction of their rate): on a B200 a quantize + attention step takes 7-9 %
- * longer than with per-slice smoothing (B1 H12 N32760 d128 and B1 H32 N8192
- * d128 causal).  Other arguments,
+ * fraction of their rate): on a B200 a quantize + attention step takes 7 %
+ * (B1 H12 N32760 d128, FP16 accumulator) to 17 % (B1 H32 N8192 d128 causal)
+ * longer than with per-slice smoothing.  Other arguments,
  * alignment and error behaviour as for the per-head calls. */
 SAGE_API sage_status sage_workspace_layout_blocksmooth(int B, int H, int N, int d, int mode, sage_ws_layout* out);
 SAGE_API sage_status sage_quantize_qkv_blocksmooth(const void* q, const void* k, const void* v, int dtype, int B,

@@ -66,7 +66,8 @@ struct Roles {
 };
 constexpr uint32_t kTmemCols = 512;
 
-template <int D, int NQ>
+// RING: the softmax warps' bias buffers (FP32 mode with a bias) are present.
+template <int D, int NQ, bool RING>
 struct Smem {
   static constexpr int kQ = 128 * D;  // one Q tile (int8)
   static constexpr int kK = 128 * D;  // one K tile (int8), rows in pair order
@@ -78,7 +79,12 @@ struct Smem {
   static constexpr int off_p = off_v + kStages * kV;  // [query tile NQ][buffer 2]
   static constexpr int off_bar = off_p + 2 * NQ * kP;
   static constexpr int off_qmx = off_bar + 256;  // fused Q: granule maxima [query tile 2][granule 4][warp 2]
-  static constexpr int bytes = off_bar + 512;
+  // per softmax warp, two bias buffers of one key tile: [half 0: 64 floats]
+  // [16 bytes of padding][half 1: 64 floats] (the padding puts the halves'
+  // 16-byte chunks in different bank groups)
+  static constexpr int kBiasBuf = 528;
+  static constexpr int off_bias = off_bar + 512;
+  static constexpr int bytes = off_bias + (RING ? 2 * 8 * NQ * kBiasBuf : 0);
   static constexpr int alloc = bytes + 1024;  // room to align the base to 1024
 };
 
@@ -107,6 +113,23 @@ enum : int {
 };
 
 SAGE_DEV float lo_half_to_float(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu))); }
+
+// 16-byte asynchronous global -> shared copies, per thread, counted in groups.
+SAGE_DEV void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+SAGE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most N of this thread's committed groups are still in flight
+template <int N>
+SAGE_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+SAGE_DEV float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
 
 // The CTA's query slice and its key/value slice, read from the special
 // registers each time (volatile: recomputed where used rather than held in
@@ -138,7 +161,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   using R = Roles<F16ACC>;
   constexpr int kNQ = R::kNQ;
   constexpr int kSoftmaxWarps = R::kSoftmaxWarps, kProducerWarp = R::kProducerWarp, kMmaWarp = R::kMmaWarp;
-  using L = Smem<D, kNQ>;
+  using L = Smem<D, kNQ, HAS_BIAS && !F16ACC>;
   // TMEM columns: S_q, O_q, and (FP16 accumulator) the two 64-key chunk partials H_c
   constexpr uint32_t kColO = F16ACC ? 128u : 256u;
   constexpr uint32_t kColH = 128u + D;
@@ -472,21 +495,37 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       // A bias row of its own per query tile (Q smoothed per block) is read
       // by this CTA alone, from DRAM: its lines (two per key half and tile)
       // are prefetched into L2 two tiles ahead.  A row shared by the slice
-      // stays in L2; the FP32 mode, which loads the bias where it is used,
-      // prefetches that row's next lines into L1 instead (measured: 5-6 %
-      // faster with the shared row, 2 % slower with the per-tile rows).
+      // stays in L2.
+      // FP32 mode: each softmax warp copies the next tile's 128 bias values
+      // (512 bytes, 16 per lane) into its own shared-memory buffer while it
+      // works on the current tile, and reads them from there.
       constexpr bool bias_prefetch = kTileBias;
-      constexpr bool bias_prefetch_l1 = HAS_BIAS && !F16ACC && !kTileBias;
+      constexpr bool kBiasRing = HAS_BIAS && !F16ACC;
+      // lane's 16 bytes of key tile jj's bias values (which start at bvec - h * 64)
+      // into this warp's buffer jj & 1
+      auto bias_copy = [&](int jj) {
+        const uint32_t ring = smem_u32(smem + L::off_bias) + (uint32_t)warp * 2 * L::kBiasBuf;
+        cp_async16(ring + (jj & 1) * L::kBiasBuf + 16 * lane + (lane >= 16 ? 16 : 0),
+                   bvec - h * 64 + (size_t)jj * bstride + 4 * lane);
+      };
       if (bias_prefetch) {
         prefetch_l2(bvec + 32 * (lane & 1));
         if (nt[q] > 1) prefetch_l2(bvec + bstride + 32 * (lane & 1));
       }
-      if (bias_prefetch_l1) prefetch_l1(bvec + 32 * (lane & 1));
+      if constexpr (kBiasRing) {
+        bias_copy(0);
+        cp_async_commit();
+      }
       for (int j = 0; ok && j < nt[q]; ++j) {
         const float2 ks = ks_next;
         if (j + 1 < nt[q]) ks_next = *reinterpret_cast<const float2*>(ksc + 2 * (j + 1));
         if (bias_prefetch && j + 2 < nt[q]) prefetch_l2(bvec + (size_t)(j + 2) * bstride + 32 * (lane & 1));
-        if (bias_prefetch_l1 && j + 1 < nt[q]) prefetch_l1(bvec + (j + 1) * 128 + 32 * (lane & 1));
+        if constexpr (kBiasRing) {
+          // buffer (j + 1) & 1 was last read for tile j - 1, by this warp
+          __syncwarp();
+          if (j + 1 < nt[q]) bias_copy(j + 1);
+          cp_async_commit();  // (an empty group on the last tile keeps the count)
+        }
         const int kbase = j * 128 + h * 64;
         // visible keys of this row among the half's 64 form the prefix c < lim
         int lim = 64;
@@ -496,7 +535,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         }
         // FP16 mode: the tile's 64 bias values, loaded before the wait for S
         // hides their latency; the FP32 mode, whose 576 threads leave no
-        // registers for it, loads them where they are used
+        // registers for it, reads them from its warp's shared-memory buffer
         constexpr int kAhead = F16ACC ? 16 : 0;
         float4 bv[HAS_BIAS && kAhead > 0 ? kAhead : 1];
         if (HAS_BIAS) {
@@ -550,10 +589,20 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
           float ma = -INFINITY, mb = -INFINITY;
           const float4* b4 = reinterpret_cast<const float4*>(kTileBias ? bvec + (size_t)j * bstride : bvec + j * 128);
+          if constexpr (kBiasRing) {
+            // this tile's copies (all but the group just committed) have landed
+            cp_async_wait<1>();
+            __syncwarp();
+          }
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
             const int c = 4 * c4;
-            const float4 bw = c4 < kAhead ? bv[c4 < kAhead ? c4 : 0] : __ldg(b4 + c4);
+            float4 bw;
+            if constexpr (kBiasRing)
+              bw = lds_f4(smem_u32(smem + L::off_bias) + (uint32_t)warp * 2 * L::kBiasBuf + (j & 1) * L::kBiasBuf +
+                          h * 272 + 16 * c4);
+            else
+              bw = c4 < kAhead ? bv[c4 < kAhead ? c4 : 0] : __ldg(b4 + c4);
             const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
                                          __fmul2_rn(make_float2(bw.x, bw.y), cl2));
             const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf),
@@ -641,6 +690,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         m = m_new;
         alpha_prev = alpha;
       }
+      if constexpr (kBiasRing) cp_async_wait<0>();  // no copy into this warp's buffers outlives the loop
       if (ok && !__all_sync(0xffffffffu, mbar_wait(&o_done[q], (nt[q] - 1) & 1, abort_flag))) ok = false;
       if (ok && F16ACC) {
         tc_fence_after();
@@ -801,7 +851,7 @@ template <int D, typename OutT, int BIAS, bool F16ACC, bool FUSED_Q>
 static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                             int BH, cudaStream_t s) {
   auto kern = attn_i8f8_kernel<D, OutT, BIAS, F16ACC, FUSED_Q>;
-  using L = Smem<D, Roles<F16ACC>::kNQ>;
+  using L = Smem<D, Roles<F16ACC>::kNQ, BIAS != 0 && !F16ACC>;
   // set on every launch: the attribute is per device, and a cached flag would
   // be shared by host threads and devices
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
