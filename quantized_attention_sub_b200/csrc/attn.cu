@@ -114,22 +114,6 @@ enum : int {
 
 SAGE_DEV float lo_half_to_float(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu))); }
 
-// 16-byte asynchronous global -> shared copies, per thread, counted in groups.
-SAGE_DEV void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-SAGE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// wait until at most N of this thread's committed groups are still in flight
-template <int N>
-SAGE_DEV void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-SAGE_DEV float4 lds_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
-               : "memory");
-  return v;
-}
 
 // The CTA's query slice and its key/value slice, read from the special
 // registers each time (volatile: recomputed where used rather than held in

@@ -148,7 +148,8 @@ struct SmemF {
   static constexpr int off_bar = off_p + 2 * kTile;
   static constexpr int off_x = off_bar + 256;  // [parity 2][half 2][row 128] floats
   static constexpr int off_rtab = off_x + 2 * 2 * 128 * 4;  // [128] P~ block reciprocals
-  static constexpr int bytes = off_rtab + 128 * 4;
+  static constexpr int off_bias = off_rtab + 128 * 4;         // [softmax warp 8][buffer 2][64 floats]
+  static constexpr int bytes = off_bias + 8 * 2 * 256;
   static constexpr int alloc = bytes + 1024;
 };
 static_assert(SmemF::off_k % 1024 == 0 && SmemF::off_v % 1024 == 0 && SmemF::off_p % 1024 == 0, "tile alignment");
@@ -373,7 +374,20 @@ __global__ void __launch_bounds__(kThreadsF, 2)
     const int swz = (r >> 1) & 3;  // 64-byte swizzle of this row's 16-byte chunks
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // With Q smoothing each softmax warp copies the next key tile's 64 bias
+    // values of its key half (256 bytes, 16 per lane of the first 16) into
+    // its own shared-memory buffer while it works on the current tile.
+    const uint32_t bring = smem_u32(smem + L::off_bias) + (uint32_t)warp * 512;
+    if constexpr (HAS_BIAS) {
+      if (lane < 16) cp_async16(bring + 16 * lane, bvec + 4 * lane);
+      cp_async_commit();
+    }
     for (int j = 0; j < T; ++j) {
+      if constexpr (HAS_BIAS) {
+        __syncwarp();  // buffer (j + 1) & 1 was last read for tile j - 1
+        if (j + 1 < T && lane < 16) cp_async16(bring + ((j + 1) & 1) * 256 + 16 * lane, bvec + (j + 1) * 128 + 4 * lane);
+        cp_async_commit();
+      }
       const int kbase = j * 128 + h * 64;
       int lim = 64;
       if (kbase + 63 >= a.N || (a.causal && j == qt)) {
@@ -410,12 +424,15 @@ __global__ void __launch_bounds__(kThreadsF, 2)
         }
         mt = __fmul_rn(fmaxf(ga, gb), kf);
       } else {
-        const float4* b4 = reinterpret_cast<const float4*>(bvec + j * 128);
+        // this tile's copies (all but the group just committed) have landed
+        cp_async_wait<1>();
+        __syncwarp();
+        const uint32_t bsm = bring + (j & 1) * 256;
         const float2 cl2 = make_float2(a.c_log2, a.c_log2);
         float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 bv = __ldg(b4 + c4);
+          const float4 bv = lds_f4(bsm + 16 * c4);
           const int c = 4 * c4;
           const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
                                        __fmul2_rn(make_float2(bv.x, bv.y), cl2));
@@ -523,6 +540,7 @@ __global__ void __launch_bounds__(kThreadsF, 2)
       l = __fadd_rn(__fmul_rn(alpha, l), (sa.x + sa.y) + (sb.x + sb.y));
       m = m_new;
     }
+    if constexpr (HAS_BIAS) cp_async_wait<0>();  // no copy into this warp's buffers outlives the loop
     if (ok && !__all_sync(0xffffffffu, mbar_wait(o_done, (T - 1) & 1, abort_flag))) ok = false;
     if (ok) {
       const int jx = T;
