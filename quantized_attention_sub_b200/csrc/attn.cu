@@ -573,24 +573,42 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
           float ma = -INFINITY, mb = -INFINITY;
           const float4* b4 = reinterpret_cast<const float4*>(kTileBias ? bvec + (size_t)j * bstride : bvec + j * 128);
+          const uint32_t bbuf = smem_u32(smem + L::off_bias) + (uint32_t)warp * 2 * L::kBiasBuf + (j & 1) * L::kBiasBuf;
           if constexpr (kBiasRing) {
             // this tile's copies (all but the group just committed) have landed
             cp_async_wait<1>();
+            if constexpr (kTileBias) {
+              // each lane turns its own 16 bytes into bias * log2(e)/sqrt(d)
+              // (the same rounded products the loop below would form), once
+              // for the warp (measured: 2 % faster with the per-tile rows,
+              // 1.5 % slower with the shared row, whose loop keeps the multiply)
+              const uint32_t mine = bbuf + 16 * lane + (lane >= 16 ? 16 : 0);
+              const float4 b = lds_f4(mine);
+              const float2 lo = __fmul2_rn(make_float2(b.x, b.y), cl2), hi = __fmul2_rn(make_float2(b.z, b.w), cl2);
+              sts_f4(mine, make_float4(lo.x, lo.y, hi.x, hi.y));
+            }
             __syncwarp();
           }
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
             const int c = 4 * c4;
-            float4 bw;
-            if constexpr (kBiasRing)
-              bw = lds_f4(smem_u32(smem + L::off_bias) + (uint32_t)warp * 2 * L::kBiasBuf + (j & 1) * L::kBiasBuf +
-                          h * 272 + 16 * c4);
-            else
-              bw = c4 < kAhead ? bv[c4 < kAhead ? c4 : 0] : __ldg(b4 + c4);
-            const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf),
-                                         __fmul2_rn(make_float2(bw.x, bw.y), cl2));
-            const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf),
-                                         __fmul2_rn(make_float2(bw.z, bw.w), cl2));
+            float2 bl, bh;  // bias * log2(e)/sqrt(d) of keys c .. c + 3
+            if constexpr (kBiasRing) {
+              const float4 bw = lds_f4(bbuf + h * 272 + 16 * c4);
+              if constexpr (kTileBias) {
+                bl = make_float2(bw.x, bw.y);
+                bh = make_float2(bw.z, bw.w);
+              } else {
+                bl = __fmul2_rn(make_float2(bw.x, bw.y), cl2);
+                bh = __fmul2_rn(make_float2(bw.z, bw.w), cl2);
+              }
+            } else {
+              const float4 bw = c4 < kAhead ? bv[c4 < kAhead ? c4 : 0] : __ldg(b4 + c4);
+              bl = __fmul2_rn(make_float2(bw.x, bw.y), cl2);
+              bh = __fmul2_rn(make_float2(bw.z, bw.w), cl2);
+            }
+            const float2 ta = __ffma2_rn(make_float2(u2f(sr[c]), u2f(sr[c + 1])), make_float2(kf, kf), bl);
+            const float2 tb = __ffma2_rn(make_float2(u2f(sr[c + 2]), u2f(sr[c + 3])), make_float2(kf, kf), bh);
             sr[c] = f2u(ta.x);
             sr[c + 1] = f2u(ta.y);
             sr[c + 2] = f2u(tb.x);
