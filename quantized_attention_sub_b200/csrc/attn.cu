@@ -66,7 +66,7 @@ struct Roles {
 };
 constexpr uint32_t kTmemCols = 512;
 
-// RING: the softmax warps' bias buffers (FP32 mode with a bias) are present.
+// RING: the softmax warps' bias buffers (kernels with a bias) are present.
 template <int D, int NQ, bool RING>
 struct Smem {
   static constexpr int kQ = 128 * D;  // one Q tile (int8)
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
   using R = Roles<F16ACC>;
   constexpr int kNQ = R::kNQ;
   constexpr int kSoftmaxWarps = R::kSoftmaxWarps, kProducerWarp = R::kProducerWarp, kMmaWarp = R::kMmaWarp;
-  using L = Smem<D, kNQ, HAS_BIAS && !F16ACC>;
+  using L = Smem<D, kNQ, HAS_BIAS>;
   // TMEM columns: S_q, O_q, and (FP16 accumulator) the two 64-key chunk partials H_c
   constexpr uint32_t kColO = F16ACC ? 128u : 256u;
   constexpr uint32_t kColH = 128u + D;
@@ -480,11 +480,11 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
       // by this CTA alone, from DRAM: its lines (two per key half and tile)
       // are prefetched into L2 two tiles ahead.  A row shared by the slice
       // stays in L2.
-      // FP32 mode: each softmax warp copies the next tile's 128 bias values
-      // (512 bytes, 16 per lane) into its own shared-memory buffer while it
-      // works on the current tile, and reads them from there.
+      // Each softmax warp copies the next tile's 128 bias values (512 bytes,
+      // 16 per lane) into its own shared-memory buffer while it works on the
+      // current tile, and reads them from there.
       constexpr bool bias_prefetch = kTileBias;
-      constexpr bool kBiasRing = HAS_BIAS && !F16ACC;
+      constexpr bool kBiasRing = HAS_BIAS;
       // lane's 16 bytes of key tile jj's bias values (which start at bvec - h * 64)
       // into this warp's buffer jj & 1
       auto bias_copy = [&](int jj) {
@@ -516,16 +516,6 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         if (kbase + 63 >= a.Nk || (a.causal && kbase + 63 > row + a.koff)) {
           lim = min(lim, a.Nk - kbase);
           if (a.causal) lim = min(lim, row + a.koff - kbase + 1);
-        }
-        // FP16 mode: the tile's 64 bias values, loaded before the wait for S
-        // hides their latency; the FP32 mode, whose 576 threads leave no
-        // registers for it, reads them from its warp's shared-memory buffer
-        constexpr int kAhead = F16ACC ? 16 : 0;
-        float4 bv[HAS_BIAS && kAhead > 0 ? kAhead : 1];
-        if (HAS_BIAS) {
-          const float4* b4 = reinterpret_cast<const float4*>(kTileBias ? bvec + (size_t)j * bstride : bvec + j * 128);
-#pragma unroll
-          for (int c4 = 0; c4 < kAhead; ++c4) bv[c4] = __ldg(b4 + c4);
         }
         // warp-uniform outcome: tcgen05.ld below is a warp-collective instruction
         if (!__all_sync(0xffffffffu, mbar_wait(&s_full[q], j & 1, abort_flag))) {
@@ -572,7 +562,6 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
         } else {
           const float2 cl2 = make_float2(a.c_log2, a.c_log2);
           float ma = -INFINITY, mb = -INFINITY;
-          const float4* b4 = reinterpret_cast<const float4*>(kTileBias ? bvec + (size_t)j * bstride : bvec + j * 128);
           const uint32_t bbuf = smem_u32(smem + L::off_bias) + (uint32_t)warp * 2 * L::kBiasBuf + (j & 1) * L::kBiasBuf;
           if constexpr (kBiasRing) {
             // this tile's copies (all but the group just committed) have landed
@@ -593,17 +582,11 @@ __global__ void __launch_bounds__(Roles<F16ACC>::kThreads, 1)
           for (int c4 = 0; c4 < 16; ++c4) {
             const int c = 4 * c4;
             float2 bl, bh;  // bias * log2(e)/sqrt(d) of keys c .. c + 3
-            if constexpr (kBiasRing) {
-              const float4 bw = lds_f4(bbuf + h * 272 + 16 * c4);
-              if constexpr (kTileBias) {
-                bl = make_float2(bw.x, bw.y);
-                bh = make_float2(bw.z, bw.w);
-              } else {
-                bl = __fmul2_rn(make_float2(bw.x, bw.y), cl2);
-                bh = __fmul2_rn(make_float2(bw.z, bw.w), cl2);
-              }
+            const float4 bw = lds_f4(bbuf + h * 272 + 16 * c4);
+            if constexpr (kTileBias) {
+              bl = make_float2(bw.x, bw.y);
+              bh = make_float2(bw.z, bw.w);
             } else {
-              const float4 bw = c4 < kAhead ? bv[c4 < kAhead ? c4 : 0] : __ldg(b4 + c4);
               bl = __fmul2_rn(make_float2(bw.x, bw.y), cl2);
               bh = __fmul2_rn(make_float2(bw.z, bw.w), cl2);
             }
@@ -853,7 +836,7 @@ template <int D, typename OutT, int BIAS, bool F16ACC, bool FUSED_Q>
 static cudaError_t run_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                             int BH, cudaStream_t s) {
   auto kern = attn_i8f8_kernel<D, OutT, BIAS, F16ACC, FUSED_Q>;
-  using L = Smem<D, Roles<F16ACC>::kNQ, BIAS != 0 && !F16ACC>;
+  using L = Smem<D, Roles<F16ACC>::kNQ, BIAS != 0>;
   // set on every launch: the attribute is per device, and a cached flag would
   // be shared by host threads and devices
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
