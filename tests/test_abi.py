@@ -124,3 +124,24 @@ def test_blocksmooth_layout_holds_a_row_per_block(lib):
     st = lib.sage_attn_fwd_blocksmooth(vp(4096), vp(4096), vp(4096), vp(4096), 1, 2, 300, 128, 0, 2, 0, vp(4096),
                                        1 << 30, vp(0))
     assert st == api.SAGE_ERR_UNSUPPORTED
+
+
+def test_blocksmooth_bias_view_follows_the_key_tile_major_layout(lib):
+    """The workspace stores block b's bias at key j at element
+    ((bh * nkt + j // 128) * nblk + b) * 128 + j % 128; the binding's q_bias
+    view reads it back as [bh, b, j]."""
+    import torch
+    B, H, N, d, mode = 1, 2, 300, 64, 0
+    L = api.sage_workspace_layout_blocksmooth(B, H, N, d, mode)
+    ws = torch.zeros(L.total, dtype=torch.uint8)
+    BH, Np = B * H, (N + 127) // 128 * 128
+    nb = Np // 128
+    flat = ws[L.q_bias:L.q_bias + BH * nb * Np * 4].view(torch.float32)
+    for bh in range(BH):
+        for b in range(nb):
+            for j in range(Np):
+                flat[((bh * nb + j // 128) * nb + b) * 128 + j % 128] = bh * 1e6 + b * 1e4 + j
+    v = api.ws_views_blocksmooth(ws, B, H, N, d, mode)["q_bias"]
+    want = (torch.arange(BH)[:, None, None] * 1e6 + torch.arange(nb)[None, :, None] * 1e4
+            + torch.arange(Np)[None, None, :]).float()
+    assert torch.equal(v, want)
